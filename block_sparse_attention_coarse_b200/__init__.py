@@ -1,0 +1,254 @@
+"""Python binding of the ISA (In-context Sparse Attention) forward library.
+
+Thin ctypes layer over ``libisa.so`` (entry points in include/isa.h): it
+marshals torch tensor pointers, sizes and the current CUDA stream and turns
+status codes into exceptions.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback -- importing
+works without a GPU, but any call fails loudly if the library or a CUDA
+device is missing.
+
+The method is the sparse attention of "LIVEditor-14B: Lightning Unified
+Video Editing via In-Context Sparse Attention" (paper.rainbus.top summary,
+"Method steps in detail"):
+  plan(...)    steps (1)-(3) + the exact-block choice of step (5)
+  forward(...) steps (4)-(6), sharp and flat query blocks in one launch
+  dense(...)   the full attention that ISA replaces
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libisa.so")
+
+ISA_OK = 0
+ISA_ERR_INVALID_ARG = 1
+ISA_ERR_UNSUPPORTED = 2
+ISA_ERR_WORKSPACE = 3
+ISA_ERR_CUDA = 4
+ISA_ERR_DEVICE_TIMEOUT = 5
+
+# every entry point declared in include/isa.h
+EXPORTS = (
+    "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
+    "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
+)
+
+
+class IsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"isa status {status}: {message}")
+        self.status = status
+
+
+class Params(ctypes.Structure):
+    """isa_params: shapes, the three ratios and the softmax scale (<= 0: 1/sqrt(D))."""
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("L_src", ctypes.c_int32), ("L_ctx", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("alpha_s", ctypes.c_float), ("alpha_f", ctypes.c_float), ("alpha_ns", ctypes.c_float),
+                ("scale", ctypes.c_float)]
+
+    def __repr__(self) -> str:
+        return ("Params(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")")
+
+
+class _PlanView(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T_src", "T_ctx", "T", "K_sel", "T_kv", "n_flat", "n_sharp", "n_exact", "T_kv_pad",
+                 "bitmap_words")] + \
+               [(n, ctypes.c_void_p) for n in
+                ("Qc", "Kc", "Vc", "imp", "ctx_sel", "kept", "energy", "sharp_ids", "flat_ids", "exact",
+                 "exact_bits", "Kp", "Vp", "status")]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads libisa.so once.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise IsaError(ISA_ERR_CUDA, f"{LIB_PATH} is missing; build it with "
+                                     "`python -m block_sparse_attention_coarse_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(Params)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.isa_plan_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.isa_plan.argtypes = [P, vp, vp, vp, vp, sz, vp]
+    lib.isa_plan_view_get.argtypes = [P, vp, sz, ctypes.POINTER(_PlanView)]
+    lib.isa_forward.argtypes = [P, vp, vp, vp, vp, sz, vp, vp, vp]
+    lib.isa_dense.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.isa_last_error.restype = ctypes.c_char_p
+    lib.isa_version.restype = ctypes.c_char_p
+    lib.isa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.isa_set_fault_injection.argtypes = [ctypes.c_int32]
+    for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
+                 "isa_set_wait_timeout_ns", "isa_set_fault_injection"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != ISA_OK:
+        raise IsaError(status, load_library().isa_last_error().decode())
+
+
+def make_params(B: int, H: int, D: int, L_src: int, L_ctx: int, block: int = 64, alpha_s: float = 0.125,
+                alpha_f: float = 0.5, alpha_ns: float = 0.0625, scale: float = 0.0) -> Params:
+    return Params(B, H, D, L_src, L_ctx, block, alpha_s, alpha_f, alpha_ns, scale)
+
+
+def version() -> str:
+    return load_library().isa_version().decode()
+
+
+def workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().isa_plan_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params) -> None:
+    shape = (p.B, p.H, p.L_src + p.L_ctx, p.D)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise IsaError(ISA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise IsaError(ISA_ERR_INVALID_ARG, f"{name} must be contiguous bfloat16 {shape}, "
+                                                f"got {t.dtype} {tuple(t.shape)}")
+
+
+def alloc_workspace(p: Params, device=None) -> torch.Tensor:
+    return torch.empty(workspace_size(p), dtype=torch.uint8, device=device or "cuda")
+
+
+def plan(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,
+         stream=None) -> torch.Tensor:
+    """Runs the planning kernels; returns the workspace holding the plan."""
+    _check_qkv(q, k, v, p)
+    if ws is None:
+        ws = alloc_workspace(p, q.device)
+    _check(load_library().isa_plan(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), ws.data_ptr(),
+                                   ws.numel(), _stream(stream)))
+    return ws
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ws: torch.Tensor, p: Params,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Sparse attention with a plan from `plan`; returns out [B,H,L,D] bf16."""
+    _check_qkv(q, k, v, p)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().isa_forward(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), ws.data_ptr(),
+                                      ws.numel(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                      _stream(stream)))
+    return out
+
+
+def dense(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, out: Optional[torch.Tensor] = None,
+          lse: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense softmax attention over all L tokens with the same kernel machinery."""
+    _check_qkv(q, k, v, p)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().isa_dense(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None,
+                                    status.data_ptr() if status is not None else None, _stream(stream)))
+    return out
+
+
+def plan_view(p: Params, ws: torch.Tensor) -> Dict[str, object]:
+    """Sizes of the plan and CUDA tensor views of every plan array in `ws`."""
+    view = _PlanView()
+    _check(load_library().isa_plan_view_get(ctypes.byref(p), ws.data_ptr(), ws.numel(), ctypes.byref(view)))
+    BH = p.B * p.H
+    base = ws.data_ptr()
+
+    def arr(ptr, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        off = ptr - base
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    v = view
+    out: Dict[str, object] = {f: getattr(v, f) for f in
+                              ("T_src", "T_ctx", "T", "K_sel", "T_kv", "n_flat", "n_sharp", "n_exact", "T_kv_pad",
+                               "bitmap_words")}
+    out.update(
+        Qc=arr(v.Qc, torch.float32, (BH, v.T, p.D)), Kc=arr(v.Kc, torch.float32, (BH, v.T, p.D)),
+        Vc=arr(v.Vc, torch.float32, (BH, v.T, p.D)), imp=arr(v.imp, torch.float32, (BH, v.T_ctx)),
+        ctx_sel=arr(v.ctx_sel, torch.int32, (BH, v.K_sel)), kept=arr(v.kept, torch.int32, (BH, v.T_kv)),
+        energy=arr(v.energy, torch.float32, (BH, v.T)),
+        sharp_ids=arr(v.sharp_ids, torch.int32, (BH, v.n_sharp)),
+        flat_ids=arr(v.flat_ids, torch.int32, (BH, v.n_flat)),
+        exact=arr(v.exact, torch.int32, (BH, v.n_flat, v.n_exact)),
+        exact_bits=arr(v.exact_bits, torch.int32, (BH, v.n_flat, v.bitmap_words)),
+        Kp=arr(v.Kp, torch.bfloat16, (BH, v.T_kv_pad, p.D)), Vp=arr(v.Vp, torch.bfloat16, (BH, v.T_kv_pad, p.D)),
+        status=arr(v.status, torch.int32, (1,)),
+    )
+    return out
+
+
+def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,
+                  device=None) -> torch.Tensor:
+    """The user-level call: plan + forward.  CUDA inputs stay on the device;
+    CPU inputs (pinned for overlap) are copied in and the output is copied
+    back to a pinned CPU tensor on the current stream."""
+    if q.is_cuda:
+        ws = plan(q, k, v, p, ws)
+        return forward(q, k, v, ws, p)
+    dev = torch.device(device or "cuda")
+    qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    ws = plan(qd, kd, vd, p, ws)
+    od = forward(qd, kd, vd, ws, p)
+    out = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+    out.copy_(od, non_blocking=True)
+    return out
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _check(load_library().isa_set_wait_timeout_ns(int(ns)))
+
+
+def set_fault_injection(mode: int) -> None:
+    _check(load_library().isa_set_fault_injection(int(mode)))
+
+
+def executed_flops(p: Params, view: Dict[str, object]) -> float:
+    """Algorithmic work of one ISA forward from a plan view copied to the
+    host: 4*D per (query token, key column) pair -- an exact key token is one
+    column, a pooled block one column -- plus 2*T*T*D per head for the
+    coarse scores."""
+    import numpy as np
+    b = p.block
+    T_src, T = int(view["T_src"]), int(view["T"])
+    cnt = np.array([min(b, p.L_src - j * b) for j in range(T_src)] +
+                   [min(b, p.L_ctx - c * b) for c in range(T - T_src)], np.float64)
+    kept = view["kept"].cpu().numpy()
+    sharp = view["sharp_ids"].cpu().numpy()
+    flat = view["flat_ids"].cpu().numpy()
+    exact = view["exact"].cpu().numpy()
+    T_kv, n_ex = int(view["T_kv"]), int(view["n_exact"])
+    total = 0.0
+    for h in range(kept.shape[0]):
+        kv_tokens = cnt[kept[h]].sum()
+        total += cnt[sharp[h]].sum() * kv_tokens
+        if flat.shape[1]:
+            ex_tok = cnt[kept[h][exact[h]]].sum(axis=1) if n_ex else np.zeros(flat.shape[1])
+            total += float((cnt[flat[h]] * (ex_tok + (T_kv - n_ex))).sum())
+    return 4.0 * p.D * total + 2.0 * T * T * p.D * kept.shape[0]

@@ -1,0 +1,474 @@
+// Attention kernel of the ISA forward pass for sm_100a: steps (4)-(6) of
+// "Method steps in detail" on the paper.rainbus.top summary card of
+// "LIVEditor-14B: Lightning Unified Video Editing via In-Context Sparse
+// Attention", with the 0th-order Taylor term of its "0th-order Taylor
+// approximate attention" section, and the dense attention it replaces.
+//
+// One persistent launch walks a list of work items.  An item is a 128-row
+// query tile made of G = 128/R query blocks of R = b rows and a sequence of
+// 128-column KV tiles, each made of G sub-blocks of R rows:
+//   sharp item : G sharp blocks of one head; KV tiles run over the kept
+//                blocks (source blocks, then the selected context blocks)
+//   flat item  : G flat blocks of one head; first n_exact tiles whose
+//                sub-block g is exact block j of query block g (block-diagonal
+//                mask), then the pooled tiles: 128 rows of the head's kept
+//                pooled keys/values (Kp, Vp) with logit bias log2(n_j) and the
+//                row's own exact blocks masked out
+//   dense item : 128 consecutive query tokens against all L tokens
+// All tiles of an item update one online-softmax state per query row, so the
+// exact and the pooled terms share one normaliser.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0 lane 0 : TMA producer (Q tile double-buffered, K/V in kNS stages)
+//   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma
+//   warps 2..5    : softmax / correction / epilogue, thread = query row
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256, 256+D).  P (bf16)
+// overwrites the first 64 columns of its S buffer and feeds the P.V MMA as the
+// A operand straight from TMEM.
+#include "isa_common.cuh"
+
+namespace isa {
+
+constexpr int kThreads = 192;
+constexpr int kNS = 2;              // K/V pipeline stages
+constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
+
+template <int D, int R>
+struct Cfg {
+  static constexpr int G = 128 / R;
+  static constexpr int NCH = D / 64;                       // 64-column chunks of a row
+  static constexpr uint32_t CHUNK = 128 * 128;             // 128 rows x 128 bytes
+  static constexpr uint32_t TILE = 128 * D * 2;            // one 128-row tile
+  static constexpr uint32_t BOX = R * 128;                 // one TMA box
+  static constexpr uint32_t Q_OFF = 0;                     // 2 buffers
+  static constexpr uint32_t K_OFF = 2 * TILE;
+  static constexpr uint32_t V_OFF = K_OFF + kNS * TILE;
+  // + 1024 alignment slack; at least 120 KB so that only one CTA (and one
+  // 512-column TMEM allocation) fits on an SM
+  static constexpr uint32_t SMEM_USED = V_OFF + kNS * TILE + 1024;
+  static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0);
+  static constexpr uint32_t ID_O = idesc_bf16_f32(128, D, 1);
+};
+
+struct Item {
+  int bh, kind;     // kind: 0 dense, 1 sharp, 2 flat
+  int slot0;        // first slot in the sharp/flat list, or the q tile (dense)
+  int ntiles;
+};
+
+template <int G>
+__device__ __forceinline__ Item decode_item(const AttnArgs& a, int it) {
+  Item r;
+  if (a.mode == 1) {
+    r.kind = 0;
+    r.bh = it / a.q_tiles;
+    r.slot0 = it % a.q_tiles;
+    r.ntiles = (a.L + 127) / 128;
+  } else if (it < a.BH * a.items_sharp) {
+    r.kind = 1;
+    r.bh = it / a.items_sharp;
+    r.slot0 = (it % a.items_sharp) * G;
+    r.ntiles = (a.T_kv + G - 1) / G;
+  } else {
+    it -= a.BH * a.items_sharp;
+    r.kind = 2;
+    r.bh = it / a.items_flat;
+    r.slot0 = (it % a.items_flat) * G;
+    r.ntiles = a.n_exact + (a.T_kv + 127) / 128;
+  }
+  return r;
+}
+
+// (token start, valid rows) of query slot g of an item.
+template <int R>
+__device__ __forceinline__ int2 q_span(const AttnArgs& a, const Item& I, int g) {
+  if (I.kind == 0) {
+    const int s = I.slot0 * 128 + g * R;
+    return make_int2(s, max(0, min(R, a.L - s)));
+  }
+  const int idx = I.slot0 + g;
+  const int n = I.kind == 1 ? a.n_sharp : a.n_flat;
+  if (idx >= n) return make_int2(0, 0);
+  const int id = (I.kind == 1 ? a.sharp : a.flat)[(size_t)I.bh * n + idx];
+  return block_span(id, a.L_src, a.L_ctx, a.b, a.T_src);
+}
+
+// (start row, valid rows, pooled?) of KV sub-block g of tile j.  Token rows
+// are positions in [0, L); pooled rows are positions in the head's Kp/Vp.
+template <int R, int G>
+__device__ __forceinline__ int3 kv_span(const AttnArgs& a, const Item& I, int j, int g) {
+  if (I.kind == 0) {
+    const int s = j * 128 + g * R;
+    return make_int3(s, max(0, min(R, a.L - s)), 0);
+  }
+  if (I.kind == 1) {
+    const int kk = j * G + g;
+    if (kk >= a.T_kv) return make_int3(0, 0, 0);
+    const int2 sp = block_span(a.kept[(size_t)I.bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src);
+    return make_int3(sp.x, sp.y, 0);
+  }
+  if (j < a.n_exact) {
+    const int f = I.slot0 + g;
+    if (f >= a.n_flat) return make_int3(0, 0, 0);
+    const int kk = a.exact[((size_t)I.bh * a.n_flat + f) * a.n_exact + j];
+    const int2 sp = block_span(a.kept[(size_t)I.bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src);
+    return make_int3(sp.x, sp.y, 0);
+  }
+  const int r0 = (j - a.n_exact) * 128 + g * R;
+  return make_int3(r0, max(0, min(R, a.T_kv - r0)), 1);
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                const __grid_constant__ CUtensorMap tm_vp, const AttnArgs a) {
+  using C = Cfg<D, R>;
+  constexpr int G = C::G;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kNS], k_empty[kNS], v_full[kNS], v_empty[kNS];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done, o_free, drain_bar, inject_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    mbar_init(&pv_done, 1);
+    mbar_init(&o_free, 128);
+    mbar_init(&drain_bar, 1);
+    mbar_init(&inject_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_kp);
+    tma_prefetch_desc(&tm_vp);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const WaitCtl wc{&abort_flag, a.status, a.timeout_ns};
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int q_cnt[2] = {0, 0}, k_cnt[kNS], v_cnt[kNS];
+    for (int i = 0; i < kNS; ++i) k_cnt[i] = v_cnt[i] = 0;
+    int n = 0, t = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      const int qb = n & 1;
+      if (n >= 2 && !mbar_wait(&q_empty[qb], ((n >> 1) - 1) & 1, wc)) break;
+      mbar_arrive_expect_tx(&q_full[qb], C::TILE);
+      ++q_cnt[qb];
+      for (int g = 0; g < G; ++g) {
+        const int2 sp = q_span<R>(a, I, g);
+        const int row = I.bh * a.L + (sp.y > 0 ? sp.x : 0);
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_2d(sgen + C::Q_OFF + qb * C::TILE + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[qb]);
+      }
+      for (int j = 0; j < I.ntiles; ++j, ++t) {
+        const int s = t % kNS;
+        if (t >= kNS && !mbar_wait(&k_empty[s], ((t / kNS) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        int rows[G];
+        bool pooled = false;
+        for (int g = 0; g < G; ++g) {
+          const int3 sp = kv_span<R, G>(a, I, j, g);
+          pooled = sp.z != 0;
+          rows[g] = pooled ? I.bh * a.T_kv_pad + sp.x : I.bh * a.L + (sp.y > 0 ? sp.x : 0);
+        }
+        const CUtensorMap* mk = pooled ? &tm_kp : &tm_k;
+        const CUtensorMap* mv = pooled ? &tm_vp : &tm_v;
+        mbar_arrive_expect_tx(&k_full[s], C::TILE);
+        ++k_cnt[s];
+        for (int g = 0; g < G; ++g)
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_2d(sgen + C::K_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, mk, c * 64, rows[g], &k_full[s]);
+        if (t >= kNS && !mbar_wait(&v_empty[s], ((t / kNS) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[s], C::TILE);
+        ++v_cnt[s];
+        for (int g = 0; g < G; ++g)
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_2d(sgen + C::V_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, mv, c * 64, rows[g], &v_full[s]);
+      }
+    }
+    // let every copy in flight land before the CTA can exit
+    for (int i = 0; i < 2; ++i)
+      if (q_cnt[i]) mbar_wait_drain(&q_full[i], (q_cnt[i] - 1) & 1, a.timeout_ns);
+    for (int i = 0; i < kNS; ++i) {
+      if (k_cnt[i]) mbar_wait_drain(&k_full[i], (k_cnt[i] - 1) & 1, a.timeout_ns);
+      if (v_cnt[i]) mbar_wait_drain(&v_full[i], (v_cnt[i] - 1) & 1, a.timeout_ns);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    bool issued = false, ok = true;
+    if (a.inject) ok = mbar_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
+    int n = 0, t = 0;
+    const uint32_t tS = tmem, tO = tmem + 256;
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      const int qb = n & 1;
+      if (!mbar_wait(&q_full[qb], (n >> 1) & 1, wc)) break;
+      tc_fence_after();
+      const uint32_t qaddr = sbase + C::Q_OFF + qb * C::TILE;
+      for (int j = 0; ok && j <= I.ntiles; ++j, ++t) {
+        if (j < I.ntiles) {
+          // S_t = Q K_t^T into S buffer t&1
+          const int s = t % kNS;
+          if (!mbar_wait(&k_full[s], (t / kNS) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+            mma_ss(tS + (t & 1) * 128, smem_desc_sw128(qaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024),
+                   C::ID_S, ks > 0);
+          }
+          issued = true;
+          tc_commit(&s_full[t & 1]);
+          tc_commit(&k_empty[s]);
+        }
+        if (j > 0) {
+          // O (+)= P_{t-1} V_{t-1}
+          const int tp = t - 1, sp = tp % kNS;
+          const bool first = (j == 1);
+          if (!mbar_wait(&p_full[tp & 1], (tp >> 1) & 1, wc) || !mbar_wait(&v_full[sp], (tp / kNS) & 1, wc) ||
+              (first && n > 0 && !mbar_wait(&o_free, (n - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t vaddr = sbase + C::V_OFF + sp * C::TILE;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tO, tS + (tp & 1) * 128 + ks * 8, smem_desc_sw128(vaddr + ks * 2048, C::CHUNK, 1024), C::ID_O,
+                   (!first || ks > 0) ? 1u : 0u);
+          tc_commit(&v_empty[sp]);
+          tc_commit(&pv_done);
+        }
+      }
+      if (!ok) break;
+      --t;   // the loop ran one step past the last tile
+      tc_commit(&q_empty[qb]);
+    }
+    if (issued) {
+      tc_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0, a.timeout_ns);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int g_r = row / R, rr = row % R;
+    int n = 0, t = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      const int2 qs = q_span<R>(a, I, g_r);
+      const bool row_valid = rr < qs.y;
+      // pooled-tile data of this row's flat block
+      const uint32_t* rbits = nullptr;
+      int pb0 = -1, pb1 = -1;
+      float lb0 = 0.f, lb1 = 0.f;
+      const float log2b = __log2f((float)a.b);
+      if (I.kind == 2) {
+        const int f = I.slot0 + g_r;
+        if (f < a.n_flat) rbits = a.bits + ((size_t)I.bh * a.n_flat + f) * a.words;
+        if (a.L_src % a.b) {
+          pb0 = a.T_src - 1;
+          lb0 = __log2f((float)(a.L_src % a.b));
+        }
+        if ((a.L_ctx % a.b) && a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1) {
+          pb1 = a.T_kv - 1;
+          lb1 = __log2f((float)(a.L_ctx % a.b));
+        }
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < I.ntiles; ++j, ++t) {
+        const int buf = t & 1;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t >> 1) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(trow + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(trow + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(trow + buf * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(trow + buf * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        // column validity of this tile for this row
+        int cnt[G];
+        bool pooled = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int3 sp = kv_span<R, G>(a, I, j, g);
+          cnt[g] = sp.y;
+          pooled = sp.z != 0;
+        }
+        if (I.kind == 2 && !pooled) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) cnt[g] = (g == g_r) ? cnt[g] : 0;   // block-diagonal
+        }
+        tmem_wait_ld();
+        float x[128];
+        if (pooled) {
+          const int jp = j - a.n_exact;
+          uint32_t wd[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int wi = jp * 4 + w;
+            wd[w] = (rbits && wi < a.words) ? rbits[wi] : 0xFFFFFFFFu;
+          }
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int kk = jp * 128 + c;
+            const bool valid = kk < a.T_kv && !((wd[c >> 5] >> (c & 31)) & 1u);
+            const float bias = kk == pb0 ? lb0 : (kk == pb1 ? lb1 : log2b);
+            x[c] = valid ? fmaf(__uint_as_float(sr[c]), a.sl2, bias) : -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            x[c] = ((c % R) < cnt[c / R]) ? __uint_as_float(sr[c]) * a.sl2 : -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        const bool need = mx > m_run + kRescaleLog2;
+        const float m_new = need ? mx : m_run;
+        const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = need ? ex2(m_run - m_ref) : 1.f;
+        float sum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = ex2(x[c] - m_ref), p1 = ex2(x[c + 1] - m_ref);
+          sum += p0 + p1;
+          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+          pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        tmem_st32(trow + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(trow + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+          // rescale the running output once P.V of the previous tile landed
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(trow + 256 + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(trow + 256 + c0, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[buf]);
+      }
+      if (!ok) break;
+      // epilogue: wait for the last P.V, normalise, write rows in token order
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) break;
+      tc_fence_after();
+      uint32_t o[D];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(trow + 256 + c0, *reinterpret_cast<uint32_t(*)[32]>(&o[c0]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&o_free);
+      if (row_valid) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
+        uint4* dst = reinterpret_cast<uint4*>(a.out + tok * D);
+#pragma unroll
+        for (int c = 0; c < D; c += 8) {
+          uint4 w;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
+          w.x = *reinterpret_cast<uint32_t*>(&h0);
+          w.y = *reinterpret_cast<uint32_t*>(&h1);
+          w.z = *reinterpret_cast<uint32_t*>(&h2);
+          w.w = *reinterpret_cast<uint32_t*>(&h3);
+          dst[c / 8] = w;
+        }
+        if (a.lse) {
+          const float mref = m_run == -INFINITY ? 0.f : m_run;
+          a.lse[tok] = (mref + __log2f(l_run)) * 0.69314718055994531f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <int D, int R>
+static cudaError_t launch_t(const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st) {
+  using C = Cfg<D, R>;
+  static bool attr_done = false;   // per template instance; set once per process
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  attn_kernel<D, R><<<grid, kThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st) {
+  if (D == 128 && R == 64) return launch_t<128, 64>(maps, a, grid, st);
+  if (D == 128 && R == 32) return launch_t<128, 32>(maps, a, grid, st);
+  if (D == 64 && R == 64) return launch_t<64, 64>(maps, a, grid, st);
+  if (D == 64 && R == 32) return launch_t<64, 32>(maps, a, grid, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace isa

@@ -1,0 +1,326 @@
+// Shared definitions of the ISA CUDA library: plan-workspace layout and the
+// sm_100a device primitives (mbarrier with bounded waits, TMA tile loads,
+// tcgen05 MMA / TMEM access) written as inline PTX.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/isa.h"
+
+namespace isa {
+
+// ---------------------------------------------------------------------------
+// problem sizes derived from isa_params (host and device)
+// ---------------------------------------------------------------------------
+
+struct Dims {
+  int B, H, BH, D, L_src, L_ctx, L, b;
+  int T_src, T_ctx, T, K_sel, T_kv, n_flat, n_sharp, n_exact, T_kv_pad, words;
+  float scale;
+};
+
+// Byte offsets of every plan array inside the caller's workspace.
+struct PlanLayout {
+  size_t status, Qc, Kc, Vc, imp, ctx_sel, kept, energy, sharp, flat, exact, bits, Kp, Vp, total;
+};
+
+struct PlanPtrs {
+  int* status;
+  float *Qc, *Kc, *Vc, *imp, *energy;
+  int *ctx_sel, *kept, *sharp, *flat, *exact;
+  uint32_t* bits;
+  __nv_bfloat16 *Kp, *Vp;
+};
+
+// Argument block of the attention kernel (isa_attn.cu).
+struct AttnArgs {
+  int BH, L, L_src, L_ctx, b, T_src, T_ctx, T_kv, T_kv_pad, K_sel, n_sharp, n_flat, n_exact, words;
+  int mode;                  // 0 = ISA sparse, 1 = dense
+  int items_sharp, items_flat, q_tiles, total_items;
+  float sl2;                 // softmax scale * log2(e)
+  const int* kept;
+  const int* sharp;
+  const int* flat;
+  const int* exact;
+  const uint32_t* bits;
+  const int* ctx_sel;
+  __nv_bfloat16* out;
+  float* lse;
+  int* status;
+  unsigned long long timeout_ns;
+  int inject;
+};
+
+// launchers (host)
+cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
+                        cudaStream_t st);
+cudaError_t prepare_plan_kernels();
+cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
+
+constexpr int kMaxT = 8192;      // blocks per head
+constexpr int kMaxTkv = 6144;    // kept blocks per head
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// -- mbarrier ---------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Shared state of the bounded waits of one CTA.
+struct WaitCtl {
+  volatile int* abort;       // shared-memory flag: some wait of this CTA ran out
+  int* status;               // device status word (may be null)
+  uint64_t limit_ns;
+};
+
+// Waits for the phase `parity` of `bar`.  Gives up when the CTA's abort flag
+// is raised or, after limit_ns, raises it and records the timeout.  Returns
+// true when the phase completed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort) return false;
+    if (globaltimer() - t0 > w.limit_ns) {
+      *w.abort = 1;
+      if (w.status) atomicExch(w.status, (int)ISA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Same, but ignores the abort flag: used on the way out to let copies that
+// are already in flight land before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// -- TMA ----------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+// 2-D tiled load of box (x = column, y = row) into shared memory, completing
+// on `bar` with a byte count.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// -- tcgen05 ------------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Whole warp.  Writes the TMEM base address to *dst (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem], A read from tensor memory.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+#define ISA_R32(a) \
+  "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]),     \
+      "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]),        \
+      "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]),       \
+      "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
+#define ISA_W32(a) \
+  "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]),      \
+      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(a[16]), "r"(a[17]), "r"(a[18]),   \
+      "r"(a[19]), "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]), "r"(a[24]), "r"(a[25]), "r"(a[26]), "r"(a[27]),   \
+      "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
+
+// Warp-collective: thread i of the warp receives 32 consecutive 32-bit
+// columns of TMEM lane (lane_base + i) starting at the address's column.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
+      "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : ISA_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
+      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      ISA_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of an operand stored with the 128-byte
+// swizzle that TMA's SWIZZLE_128B writes: rows of 128 bytes, 8-row groups of
+// 1024 bytes.  lbo/sbo in bytes.  Bits: [0,14) start>>4, [16,30) lbo>>4,
+// [32,46) sbo>>4, [46,48) version 1, [61,64) layout 2 (128B swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B,
+// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M x N tile.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn) {
+  return (1u << 4)                       // D format f32
+         | (1u << 7)                     // A format bf16
+         | (1u << 10)                    // B format bf16
+         | ((uint32_t)b_mn << 16)        // B major
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Order-preserving map of a float to an unsigned key.
+__device__ __forceinline__ uint32_t f2ord(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp selects the k largest of key[0..n) (shared memory), ties to the
+// lower index, writing the chosen indices in ascending order to out[0..k)
+// and, when bits != nullptr, the selection as a bitmap of ceil(n/32) words.
+__device__ inline void warp_topk(const float* key, int n, int k, int* out, uint32_t* bits) {
+  const int lane = threadIdx.x & 31;
+  if (k >= n) {
+    for (int i = lane; i < n; i += 32) out[i] = i;
+    if (bits)
+      for (int w = lane; w < (n + 31) / 32; w += 32) {
+        int rem = n - w * 32;
+        bits[w] = rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u);
+      }
+    return;
+  }
+  uint32_t t = 0;
+  if (k > 0) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = t | (1u << bit);
+      int c = 0;
+      for (int i = lane; i < n; i += 32) c += f2ord(key[i]) >= cand;
+      c = __reduce_add_sync(0xFFFFFFFFu, c);
+      if (c >= k) t = cand;
+    }
+  }
+  int gt = 0;
+  if (k > 0) {
+    for (int i = lane; i < n; i += 32) gt += f2ord(key[i]) > t;
+    gt = __reduce_add_sync(0xFFFFFFFFu, gt);
+  }
+  const int need_eq = k - gt;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base = 0, eq_seen = 0;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t o = i < n ? f2ord(key[i]) : 0u;
+    const bool valid = (i < n) && (k > 0);
+    const bool is_gt = valid && o > t;
+    const bool is_eq = valid && o == t;
+    const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, is_eq);
+    const int eq_rank = eq_seen + __popc(eqm & lt_mask);
+    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
+    const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) out[base + __popc(selm & lt_mask)] = i;
+    if (bits && lane == 0) bits[i0 >> 5] = selm;
+    base += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+}
+
+// Token span of block `id` (source blocks first, each segment blocked on its own).
+__device__ __forceinline__ int2 block_span(int id, int L_src, int L_ctx, int b, int T_src) {
+  if (id < T_src) {
+    const int s = id * b;
+    return make_int2(s, min(b, L_src - s));
+  }
+  const int s = (id - T_src) * b;
+  return make_int2(L_src + s, min(b, L_ctx - s));
+}
+
+#endif  // __CUDACC__
+
+}  // namespace isa

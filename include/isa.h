@@ -1,0 +1,161 @@
+/*
+ * isa.h -- C interface of the In-context Sparse Attention (ISA) forward pass
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method is the sparse attention of "LIVEditor-14B: Lightning Unified
+ * Video Editing via In-Context Sparse Attention" (arXiv:2605.04569), as the
+ * paper.rainbus.top summary card states it in "Method steps in detail"
+ * (steps (1)-(6)) and "Core method", with the 0th-order Taylor term of its
+ * "0th-order Taylor approximate attention" section.  The model card
+ * (Hugging Face mirror, "Highlights") describes ISA as a drop-in for the
+ * attention call of a diffusion transformer on the concatenated
+ * [source ; context] token sequence; the entry points below are that call,
+ * split into planning and attention.
+ *
+ * Conventions shared by every entry point
+ *  - Q, K, V and O are bfloat16 tensors [B, H, L, D], contiguous, on the
+ *    current CUDA device, with L = L_src + L_ctx and the context tokens
+ *    after the source tokens.  Base addresses must be 16-byte aligned.
+ *  - "device" pointers are CUDA device (or managed) memory; the caller owns
+ *    all memory and the stream.  The library allocates no device memory,
+ *    launches asynchronously on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream) and never synchronises the host.
+ *  - Argument errors are returned synchronously before anything is
+ *    launched; launch failures are returned from the launching call
+ *    (ISA_ERR_CUDA); a device-side wait that exceeded its time limit sets a
+ *    device status word (see isa_plan_view.status / isa_dense `status`) that
+ *    the caller reads after synchronising.
+ *  - isa_last_error() returns a thread-local message for the last failure.
+ *
+ * Supported shapes: D in {64, 128}; block in {32, 64}; L_src, L_ctx >= 1;
+ * B*H*L < 2^31; alpha_s in (0, 1]; alpha_f, alpha_ns in [0, 1].
+ */
+#ifndef ISA_H_
+#define ISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem description.  The three ratios are the pages' hyper-parameters
+ * (summary card "Core method"; techwalker.com section 9): alpha_s = share of
+ * context blocks kept by the pre-selection, alpha_f = share of query blocks
+ * sent to the Taylor ("flat") path, alpha_ns = share of kept KV blocks that a
+ * flat block attends exactly.  scale <= 0 selects 1/sqrt(D). */
+typedef struct isa_params {
+  int32_t B, H, D;
+  int32_t L_src, L_ctx;
+  int32_t block;
+  float alpha_s, alpha_f, alpha_ns;
+  float scale;
+} isa_params;
+
+typedef enum isa_status {
+  ISA_OK = 0,
+  ISA_ERR_INVALID_ARG = 1,     /* null pointer, misalignment, out-of-range value   */
+  ISA_ERR_UNSUPPORTED = 2,     /* valid problem outside the supported shapes        */
+  ISA_ERR_WORKSPACE = 3,       /* plan workspace too small                          */
+  ISA_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed       */
+  ISA_ERR_DEVICE_TIMEOUT = 5   /* value written to a device status word, see above  */
+} isa_status;
+
+/* Sizes of the plan and device pointers into a plan workspace.  All arrays
+ * are per head, heads ordered bh = b*H + h.  Block ids run over the T =
+ * T_src + T_ctx blocks: source blocks 0..T_src-1 cover tokens [j*b, ...),
+ * context blocks T_src..T-1 cover tokens [L_src + c*b, ...); only each
+ * segment's last block may be partial. */
+typedef struct isa_plan_view {
+  int32_t T_src, T_ctx, T;     /* blocks per segment / in total                     */
+  int32_t K_sel;               /* kept context blocks = clamp(ceil(alpha_s*T_ctx),1,T_ctx) */
+  int32_t T_kv;                /* kept KV blocks = T_src + K_sel                    */
+  int32_t n_flat, n_sharp;     /* n_flat = floor(alpha_f*T), n_sharp = T - n_flat   */
+  int32_t n_exact;             /* exact blocks per flat block = ceil(alpha_ns*T_kv) */
+  int32_t T_kv_pad;            /* rows of Kp/Vp per head (T_kv rounded up to 128)   */
+  int32_t bitmap_words;        /* 32-bit words per exact bitmap = ceil(T_kv/32)     */
+  const float* Qc;             /* [BH, T, D] fp32 pooled means (step (1))           */
+  const float* Kc;             /* [BH, T, D]                                        */
+  const float* Vc;             /* [BH, T, D]                                        */
+  const float* imp;            /* [BH, T_ctx] context importance (step (2))         */
+  const int32_t* ctx_sel;      /* [BH, K_sel] selected context blocks, ascending    */
+  const int32_t* kept;         /* [BH, T_kv] kept block ids, ascending              */
+  const float* energy;         /* [BH, T] E_i = sum_j softmax(S_i)_j^2 (step (3)); the
+                                  sharpness variance is E_i/T - 1/T^2              */
+  const int32_t* sharp_ids;    /* [BH, n_sharp] ascending block ids                 */
+  const int32_t* flat_ids;     /* [BH, n_flat] ascending block ids                  */
+  const int32_t* exact;        /* [BH, n_flat, n_exact] positions in `kept`, ascending */
+  const uint32_t* exact_bits;  /* [BH, n_flat, bitmap_words] same set as a bitmap   */
+  const uint16_t* Kp;          /* [BH, T_kv_pad, D] bf16 pooled K of kept blocks    */
+  const uint16_t* Vp;          /* [BH, T_kv_pad, D] bf16 pooled V of kept blocks    */
+  const int32_t* status;       /* device status word: ISA_OK or ISA_ERR_DEVICE_TIMEOUT */
+} isa_plan_view;
+
+/* Bytes of device workspace isa_plan needs for `p`.  Host only; launches
+ * nothing.  Returns ISA_ERR_INVALID_ARG / ISA_ERR_UNSUPPORTED for bad `p`. */
+isa_status isa_plan_workspace_size(const isa_params* p, size_t* bytes);
+
+/* Planning: steps (1)-(3) of "Method steps in detail" and the exact-block
+ * choice of step (5).  Pools Q/K/V into blocks (fp32 means of the valid
+ * tokens), computes the coarse scores S = Qc Kc^T * scale, keeps the K_sel
+ * context blocks with the largest sum of S over source query rows (ties to
+ * the lower block), ranks query blocks by E_i (descending; ties: lower block
+ * is sharper) into n_sharp sharp and n_flat flat blocks, and gives each flat
+ * block the n_exact kept blocks with the largest S (ties to the lower block).
+ *   q, k, v : device, bf16 [B,H,L,D]
+ *   ws      : device, at least isa_plan_workspace_size bytes, 256-byte
+ *             aligned; overwritten; holds the plan afterwards
+ * Launches 5 kernels on `stream`. */
+isa_status isa_plan(const isa_params* p, const void* q, const void* k, const void* v,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Fills `view` with the sizes of the plan for `p` and device pointers into
+ * `ws` (no launch, no copy; contents valid once isa_plan has run). */
+isa_status isa_plan_view_get(const isa_params* p, const void* ws, size_t ws_bytes,
+                             isa_plan_view* view);
+
+/* Sparse attention: steps (4)-(6) of "Method steps in detail".  Sharp query
+ * blocks attend exactly to every token of the kept KV blocks; flat query
+ * blocks attend exactly to the tokens of their n_exact blocks and, for every
+ * other kept block j, to one pooled key Kc_j with value Vc_j and weight n_j
+ * (logit scale*q.Kc_j + ln n_j); one online-softmax state per query row
+ * merges both parts.  Outputs go straight to token order.
+ *   q, k, v : device, bf16 [B,H,L,D] (the tensors given to isa_plan)
+ *   ws      : device, a workspace isa_plan filled for the same p, q, k, v
+ *   out     : device, bf16 [B,H,L,D]; every row is written
+ *   lse     : device fp32 [B,H,L] natural-log softmax normaliser per row, or NULL
+ * One persistent launch (tcgen05/TMEM/TMA). */
+isa_status isa_forward(const isa_params* p, const void* q, const void* k, const void* v,
+                       const void* ws, size_t ws_bytes, void* out, float* lse, void* stream);
+
+/* Dense reference attention: softmax(scale * Q K^T) V over all L tokens per
+ * head (the full attention that ISA replaces, summary card "Background" /
+ * FlashAttention baselines), with the same kernel machinery.
+ *   out    : device bf16 [B,H,L,D];  lse: device fp32 [B,H,L] or NULL
+ *   status : device int32 status word (set to ISA_OK by the call, raised to
+ *            ISA_ERR_DEVICE_TIMEOUT by a timed-out wait), or NULL */
+isa_status isa_dense(const isa_params* p, const void* q, const void* k, const void* v,
+                     void* out, float* lse, int32_t* status, void* stream);
+
+/* Thread-local description of the last error (never NULL). */
+const char* isa_last_error(void);
+
+/* Library version string, e.g. "isa-b200 0.1 sm_100a". */
+const char* isa_version(void);
+
+/* Time limit of every device-side wait of later launches, in nanoseconds
+ * (default 2e9).  A wait that runs out writes ISA_ERR_DEVICE_TIMEOUT to the
+ * status word, stops its CTA's work, drains the CTA's copies in flight and
+ * returns.  0 restores the default. */
+isa_status isa_set_wait_timeout_ns(uint64_t ns);
+
+/* Host-chosen fault injection for tests of the timeout path: mode 1 makes
+ * the attention kernels wait on a barrier that nothing arrives on, so the
+ * wait runs out; 0 turns it off.  Applies to later launches. */
+isa_status isa_set_fault_injection(int32_t mode);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ISA_H_ */

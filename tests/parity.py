@@ -1,0 +1,164 @@
+"""Comparison helpers shared by the GPU parity tests (CPU-side logic only).
+
+Index sets are compared with the margin rule of the ISA forward spec: an
+element may differ between the CUDA plan and the fp64 oracle only where its
+score lies within `margin` of the k-th / (k+1)-th boundary.  Margins, per
+set, in that set's own units:
+  context TopK       : absolute 1e-3 on imp / T_src (the mean coarse score)
+  flat exact TopK    : absolute 1e-3 on S
+  sharp/flat split   : relative 1e-3 on E_i = sum_j softmax(S_i)_j^2
+"""
+from __future__ import annotations
+
+from typing import Iterable, List, Sequence, Tuple
+
+import numpy as np
+import torch
+
+import oracle as O
+from workloads import Workload, bf16_to_f64
+
+MARGIN_CTX = 1e-3
+MARGIN_EXACT = 1e-3
+MARGIN_SPLIT_REL = 1e-3
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+
+
+def to_torch_bf16(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def oracle_params(w: Workload) -> O.Params:
+    return O.Params(D=w.D, L_src=w.L_src, L_ctx=w.L_ctx, block=w.block, alpha_s=w.alpha_s,
+                    alpha_f=w.alpha_f, alpha_ns=w.alpha_ns)
+
+
+def topk_agrees(scores: Sequence[float], k: int, chosen: Iterable[int], margin: float) -> Tuple[bool, int]:
+    """True when `chosen` is a valid top-k of `scores` under the margin rule.
+    Also returns how many chosen elements differ from the oracle's own top-k."""
+    scores = np.asarray(scores, np.float64)
+    chosen = sorted(int(c) for c in chosen)
+    n = len(scores)
+    if len(chosen) != k or len(set(chosen)) != k or any(c < 0 or c >= n for c in chosen):
+        return False, k
+    if k == 0 or k >= n:
+        return True, 0
+    order = np.lexsort((np.arange(n), -scores))
+    vk, vk1 = scores[order[k - 1]], scores[order[k]]
+    cs = set(chosen)
+    clear_in = np.nonzero(scores > vk1 + margin)[0]
+    clear_out = np.nonzero(scores < vk - margin)[0]
+    ok = all(i in cs for i in clear_in) and not any(i in cs for i in clear_out)
+    diff = len(cs.symmetric_difference(set(order[:k].tolist()))) // 2
+    return ok, diff
+
+
+def energy_from_oracle(pl: O.HeadPlan) -> np.ndarray:
+    P = O.softmax_rows(pl.S)
+    return (P ** 2).sum(axis=1)
+
+
+class HeadCheck:
+    """Outcome of comparing one head's CUDA plan with the oracle's."""
+
+    def __init__(self):
+        self.ctx_equal = True
+        self.split_moved: List[int] = []      # blocks whose sharp/flat side differs
+        self.exact_moved: List[int] = []      # flat blocks whose exact list differs
+        self.errors: List[str] = []
+
+
+def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int) -> HeadCheck:
+    """Compares plan arrays of head `h` (host numpy copies of the plan view)
+    with the oracle plan `pl` under the margin rules."""
+    r = HeadCheck()
+    T_src = pl.T_src
+    # pooled means (fp32 sums of bf16 values)
+    for name, ref in (("Qc", pl.Qc), ("Kc", pl.Kc), ("Vc", pl.Vc)):
+        got = gpu[name][h]
+        err = np.abs(got - ref).max()
+        if err > 1e-5 * max(1.0, np.abs(ref).max()):
+            r.errors.append(f"{name} max err {err:.3g}")
+    # context importance and selection
+    if np.abs(gpu["imp"][h] - pl.imp).max() > 1e-3 * max(1.0, np.abs(pl.imp).max()):
+        r.errors.append(f"imp max err {np.abs(gpu['imp'][h] - pl.imp).max():.3g}")
+    ok, diff = topk_agrees(pl.imp / T_src, len(pl.ctx_sel), gpu["ctx_sel"][h], MARGIN_CTX)
+    if not ok:
+        r.errors.append(f"ctx_sel outside margin: gpu {gpu['ctx_sel'][h].tolist()} oracle {pl.ctx_sel.tolist()}")
+    if list(gpu["ctx_sel"][h]) != sorted(gpu["ctx_sel"][h]):
+        r.errors.append("ctx_sel not ascending")
+    r.ctx_equal = np.array_equal(np.sort(gpu["ctx_sel"][h]), pl.ctx_sel)
+    kept_gpu = gpu["kept"][h]
+    if not np.array_equal(kept_gpu, np.concatenate([np.arange(T_src), T_src + np.sort(gpu["ctx_sel"][h])])):
+        r.errors.append("kept list inconsistent with ctx_sel")
+    # energy and split
+    E = energy_from_oracle(pl)
+    if np.abs(gpu["energy"][h] - E).max() > 1e-4 * E.max():
+        r.errors.append(f"energy rel err {np.abs(gpu['energy'][h] - E).max() / E.max():.3g}")
+    n_sharp = len(pl.sharp)
+    sharp_gpu = gpu["sharp_ids"][h]
+    flat_gpu = gpu["flat_ids"][h]
+    if sorted(sharp_gpu.tolist() + flat_gpu.tolist()) != list(range(pl.T)):
+        r.errors.append("sharp/flat lists are not a partition of the blocks")
+    if list(sharp_gpu) != sorted(sharp_gpu) or list(flat_gpu) != sorted(flat_gpu):
+        r.errors.append("sharp/flat lists not ascending")
+    if n_sharp and n_sharp < pl.T:
+        order = np.lexsort((np.arange(pl.T), -E))
+        boundary = 0.5 * (E[order[n_sharp - 1]] + E[order[n_sharp]])
+        ok, _ = topk_agrees(E, n_sharp, sharp_gpu, MARGIN_SPLIT_REL * boundary)
+        if not ok:
+            r.errors.append("sharp set outside margin")
+    r.split_moved = sorted(set(sharp_gpu.tolist()).symmetric_difference(pl.sharp.tolist()))
+    # exact lists, where the kept sets agree
+    if r.ctx_equal:
+        flat_pos_gpu = {int(b): i for i, b in enumerate(flat_gpu)}
+        for ro, b in enumerate(pl.flat):
+            if int(b) not in flat_pos_gpu:
+                continue
+            got = gpu["exact"][h][flat_pos_gpu[int(b)]]
+            ok, diff = topk_agrees(pl.S[b, pl.kept], pl.exact.shape[1], got, MARGIN_EXACT)
+            if not ok:
+                r.errors.append(f"exact list of block {b} outside margin")
+            if list(got) != sorted(got):
+                r.errors.append("exact list not ascending")
+            bits = gpu["exact_bits"][h][flat_pos_gpu[int(b)]].astype(np.uint32)
+            from_bits = [i for i in range(len(pl.kept)) if (bits[i // 32] >> (i % 32)) & 1]
+            if from_bits != sorted(got.tolist()):
+                r.errors.append(f"exact bitmap of block {b} disagrees with the list")
+            if diff:
+                r.exact_moved.append(int(b))
+    return r
+
+
+def compare_outputs(out_gpu: np.ndarray, out_ref: np.ndarray, rows: np.ndarray):
+    """(max-abs, mean-abs) error over the listed rows."""
+    if len(rows) == 0:
+        return 0.0, 0.0
+    d = np.abs(out_gpu[rows].astype(np.float64) - out_ref[rows])
+    return float(d.max()), float(d.mean())
+
+
+def block_rows(pl: O.HeadPlan, blocks: Iterable[int]) -> np.ndarray:
+    rows = [np.arange(pl.starts[b], pl.starts[b] + pl.counts[b]) for b in blocks]
+    return np.concatenate(rows) if rows else np.zeros(0, np.int64)
+
+
+def plan_view_host(view: dict) -> dict:
+    """Host numpy copies of a plan view's arrays."""
+    out = {}
+    for k, v in view.items():
+        if isinstance(v, torch.Tensor):
+            out[k] = v.float().cpu().numpy() if v.dtype == torch.bfloat16 else v.cpu().numpy()
+        else:
+            out[k] = v
+    return out
+
+
+def head_inputs_f64(bits_q, bits_k, bits_v, h):
+    return bf16_to_f64(bits_q[h]), bf16_to_f64(bits_k[h]), bf16_to_f64(bits_v[h])
+
+
+__all__ = ["topk_agrees", "check_head_plan", "compare_outputs", "block_rows", "plan_view_host", "oracle_params",
+           "to_torch_bf16", "head_inputs_f64", "energy_from_oracle", "MARGIN_CTX", "MARGIN_EXACT",
+           "MARGIN_SPLIT_REL", "OUT_MAX_ABS", "OUT_MEAN_ABS"]

@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/isa.h declares, validates arguments on the host and sizes the
+plan exactly as the oracle's counting rules say."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def isa():
+    from block_sparse_attention_coarse_b200 import build
+    build.build()
+    import block_sparse_attention_coarse_b200 as I
+    I.load_library()
+    return I
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "isa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:isa_status|const char\*)\s+(isa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("isa_plan", "isa_forward", "isa_dense", "isa_plan_workspace_size", "isa_plan_view_get",
+                     "isa_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(isa):
+    lib = isa.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(isa.EXPORTS)
+    assert "sm_100a" in isa.version()
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(D=96), 2), (dict(block=16), 2), (dict(alpha_s=0.0), 1), (dict(alpha_s=1.5), 1), (dict(alpha_f=-0.1), 1),
+    (dict(alpha_ns=1.01), 1), (dict(L_src=0), 1), (dict(L_ctx=-3), 1), (dict(B=0), 1),
+    (dict(scale=float("nan")), 1), (dict(H=100000, L_src=400000, L_ctx=400000), 2),
+])
+def test_invalid_params_rejected_on_host(isa, bad, status):
+    kw = dict(B=1, H=2, D=64, L_src=100, L_ctx=50, block=64, alpha_s=0.125, alpha_f=0.5, alpha_ns=0.0625)
+    kw.update(bad)
+    p = isa.make_params(**kw)
+    with pytest.raises(isa.IsaError) as e:
+        isa.workspace_size(p)
+    assert e.value.status == status
+    assert len(isa.load_library().isa_last_error()) > 0
+
+
+def fake_view(isa, p):
+    """Sizes from isa_plan_view_get; the workspace is never dereferenced."""
+    lib = isa.load_library()
+    n = isa.workspace_size(p)
+    v = isa._PlanView()
+    st = lib.isa_plan_view_get(ctypes.byref(p), ctypes.c_void_p(1 << 20), n, ctypes.byref(v))
+    assert st == 0
+    return v, n
+
+
+@pytest.mark.parametrize("L_src,L_ctx,b,a_s,a_f,a_ns", [
+    (1024, 1024, 64, 0.125, 0.5, 0.0625), (11884, 11884, 64, 0.125, 0.5, 0.0625),
+    (16384, 16384, 64, 0.125, 0.5, 0.0625), (32768, 32768, 32, 0.125, 0.5, 0.0625),
+    (100, 37, 32, 0.3, 0.7, 0.2), (5, 3, 64, 1.0, 0.0, 1.0), (65536, 65536, 64, 0.0625, 0.5, 0.03125),
+    (300, 1, 32, 0.01, 1.0, 0.0),
+])
+def test_plan_counts_follow_the_oracle_rules(isa, L_src, L_ctx, b, a_s, a_f, a_ns):
+    p = isa.make_params(1, 3, 128, L_src, L_ctx, b, a_s, a_f, a_ns)
+    v, n = fake_view(isa, p)
+    _, _, T_src, T_ctx = O.segment_blocks(L_src, L_ctx, b)
+    T = T_src + T_ctx
+    assert (v.T_src, v.T_ctx, v.T) == (T_src, T_ctx, T)
+    assert v.K_sel == O.n_select(a_s, T_ctx)
+    assert v.T_kv == T_src + v.K_sel
+    assert v.n_flat == O.n_flat_blocks(a_f, T) and v.n_sharp == T - v.n_flat
+    assert v.n_exact == O.n_exact_blocks(a_ns, v.T_kv)
+    assert v.T_kv_pad % 128 == 0 and v.T_kv_pad >= v.T_kv
+    assert v.bitmap_words == (v.T_kv + 31) // 32
+    # every array lies inside the workspace, 256-byte aligned
+    base = 1 << 20
+    for name in ("Qc", "Kc", "Vc", "imp", "ctx_sel", "kept", "energy", "sharp_ids", "flat_ids", "exact",
+                 "exact_bits", "Kp", "Vp", "status"):
+        ptr = getattr(v, name)
+        assert base <= ptr < base + n and (ptr - base) % 256 == 0, name
+
+
+def test_workspace_too_small_is_rejected(isa):
+    p = isa.make_params(1, 2, 64, 256, 256)
+    n = isa.workspace_size(p)
+    v = isa._PlanView()
+    st = isa.load_library().isa_plan_view_get(ctypes.byref(p), ctypes.c_void_p(1 << 20), n - 1, ctypes.byref(v))
+    assert st == 3
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(isa):
+    lib = isa.load_library()
+    p = isa.make_params(1, 2, 64, 256, 256)
+    n = isa.workspace_size(p)
+    st = lib.isa_plan(ctypes.byref(p), None, 1 << 20, 1 << 20, 1 << 20, n, None)
+    assert st == 1 and b"q is NULL" in lib.isa_last_error()
+    st = lib.isa_forward(ctypes.byref(p), 1 << 20, (1 << 20) + 2, 1 << 20, 1 << 20, n, 1 << 20, None, None)
+    assert st == 1 and b"aligned" in lib.isa_last_error()
+    st = lib.isa_dense(ctypes.byref(p), 1 << 20, 1 << 20, 1 << 20, None, None, None, None)
+    assert st == 1
+
+
+def test_binding_rejects_host_tensors(isa):
+    import torch
+    p = isa.make_params(1, 1, 64, 64, 64)
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(isa.IsaError):
+        isa.plan(q, q, q, p)
+
+
+def test_debug_setters(isa):
+    isa.set_wait_timeout_ns(1000)
+    isa.set_wait_timeout_ns(0)
+    isa.set_fault_injection(0)
+    with pytest.raises(isa.IsaError):
+        isa.set_fault_injection(7)
+
+
+def test_product_path_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "block_sparse_attention_coarse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "isa_oracle" not in text, f

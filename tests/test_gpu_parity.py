@@ -1,0 +1,244 @@
+"""GPU parity of the CUDA path (through the C-ABI) against the fp64 oracle.
+
+Every case draws seeded inputs from `workloads`, runs isa_plan / isa_forward
+/ isa_dense on the GPU and compares with the oracle on the same bf16 values:
+  * plan index sets: bit-exact outside the margins of tests/parity.py;
+  * outputs: max-abs <= 2e-2 and mean-abs <= 2e-3 (bf16 inputs, fp32
+    accumulation, bf16 output), on every row whose plan decisions agree;
+  * lse (natural-log softmax normaliser): abs <= 2e-2.
+Small cases are compared in full; the full-size workloads on a seeded sample
+of heads and query blocks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity import (OUT_MAX_ABS, OUT_MEAN_ABS, block_rows, check_head_plan, compare_outputs, oracle_params,
+                    plan_view_host, to_torch_bf16)
+from workloads import Workload, bf16_to_f64, generate_bits, named_workloads, sample_blocks
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def isa():
+    from block_sparse_attention_coarse_b200 import build
+    build.build()
+    import block_sparse_attention_coarse_b200 as I
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return I
+
+
+def params_of(isa, w: Workload):
+    return isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+
+
+def run_isa(isa, w: Workload, bits=None):
+    qb, kb, vb = bits if bits is not None else generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    ws = isa.plan(q, k, v, p)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device="cuda")
+    out = isa.forward(q, k, v, ws, p, lse=lse)
+    torch.cuda.synchronize()
+    view = plan_view_host(isa.plan_view(p, ws))
+    return (qb, kb, vb), out.float().cpu().numpy().reshape(w.BH, w.L, w.D), \
+        lse.cpu().numpy().reshape(w.BH, w.L), view
+
+
+def check_case(isa, w: Workload, heads=None, blocks_per_head=None, max_moved_frac=0.02):
+    bits, out, lse, view = run_isa(isa, w)
+    assert int(view["status"][0]) == 0
+    qb, kb, vb = (x.reshape(w.BH, w.L, w.D) for x in bits)
+    p = oracle_params(w)
+    heads = range(w.BH) if heads is None else heads
+    n_blocks = n_moved = 0
+    worst = (0.0, 0.0)
+    for h in heads:
+        q, k, v = bf16_to_f64(qb[h]), bf16_to_f64(kb[h]), bf16_to_f64(vb[h])
+        pl = O.plan_head(q, k, v, p)
+        r = check_head_plan(pl, view, h)
+        assert not r.errors, (h, r.errors[:5])
+        if not r.ctx_equal:
+            n_moved += pl.T
+            n_blocks += pl.T
+            continue
+        blocks = list(range(pl.T))
+        if blocks_per_head is not None:
+            g = np.random.default_rng(1000 + h)
+            blocks = sorted(g.choice(pl.T, size=min(blocks_per_head, pl.T), replace=False).tolist())
+        moved = set(r.split_moved) | set(r.exact_moved)
+        use = [b for b in blocks if b not in moved]
+        n_blocks += len(blocks)
+        n_moved += len(blocks) - len(use)
+        ref, ref_lse = O.forward_head(q, k, v, pl, p, blocks=use)
+        rows = block_rows(pl, use)
+        mx, mean = compare_outputs(out[h], ref, rows)
+        worst = (max(worst[0], mx), max(worst[1], mean))
+        assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (h, mx, mean)
+        lerr = np.abs(lse[h][rows] - ref_lse[rows]).max() if len(rows) else 0.0
+        assert lerr <= 2e-2, (h, lerr)
+    assert n_moved <= max_moved_frac * max(n_blocks, 1), (n_moved, n_blocks)
+    return worst
+
+
+# ---------------------------------------------------------------------------
+# planning only (no tensor-core kernel involved)
+# ---------------------------------------------------------------------------
+
+def test_plan_tiny_matches_oracle(isa):
+    w = named_workloads()["tiny"]
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    ws = isa.plan(q, k, v, p)
+    torch.cuda.synchronize()
+    view = plan_view_host(isa.plan_view(p, ws))
+    op = oracle_params(w)
+    for h in range(w.BH):
+        pl = O.plan_head(bf16_to_f64(qb.reshape(w.BH, w.L, w.D)[h]), bf16_to_f64(kb.reshape(w.BH, w.L, w.D)[h]),
+                         bf16_to_f64(vb.reshape(w.BH, w.L, w.D)[h]), op)
+        r = check_head_plan(pl, view, h)
+        assert not r.errors, r.errors[:5]
+
+
+@pytest.mark.parametrize("L_src,L_ctx,b,D", [(300, 150, 64, 128), (333, 97, 32, 64), (64, 20, 32, 128)])
+def test_plan_ragged_matches_oracle(isa, L_src, L_ctx, b, D):
+    w = Workload("ragged", 1, 3, D, L_src, L_ctx, block=b, alpha_s=0.3, alpha_f=0.5, alpha_ns=0.2, seed=77)
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    ws = isa.plan(q, k, v, p)
+    torch.cuda.synchronize()
+    view = plan_view_host(isa.plan_view(p, ws))
+    op = oracle_params(w)
+    for h in range(w.BH):
+        pl = O.plan_head(*(bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb)), op)
+        r = check_head_plan(pl, view, h)
+        assert not r.errors, r.errors[:5]
+        # bf16 pooled keys/values of the kept blocks, zero padding
+        Kp = view["Kp"][h]
+        assert np.abs(Kp[:len(pl.kept)] - pl.Kc[pl.kept]).max() <= 2 ** -8 * max(1, np.abs(pl.Kc).max())
+        assert np.all(Kp[len(pl.kept):] == 0)
+
+
+# ---------------------------------------------------------------------------
+# dense kernel
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L_src,L_ctx,D", [(128, 128, 128), (200, 77, 64), (1000, 536, 128)])
+def test_dense_matches_oracle(isa, L_src, L_ctx, D):
+    w = Workload("dense", 1, 2, D, L_src, L_ctx, kind="iid", seed=5)
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    out = isa.dense(q, k, v, p, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    out = out.float().cpu().numpy().reshape(w.BH, w.L, w.D)
+    lse = lse.cpu().numpy().reshape(w.BH, w.L)
+    for h in range(w.BH):
+        ref, ref_lse = O.dense_attention(*(bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb)),
+                                         1 / np.sqrt(D))
+        d = np.abs(out[h] - ref)
+        assert d.max() <= OUT_MAX_ABS and d.mean() <= OUT_MEAN_ABS, (d.max(), d.mean())
+        assert np.abs(lse[h] - ref_lse).max() <= 2e-2
+
+
+# ---------------------------------------------------------------------------
+# ISA forward, small cases in full
+# ---------------------------------------------------------------------------
+
+def test_forward_tiny(isa):
+    check_case(isa, named_workloads()["tiny"])
+
+
+SMALL = [
+    # name, B, H, D, L_src, L_ctx, b, alpha_s, alpha_f, alpha_ns
+    ("ragged128", 1, 2, 128, 300, 150, 64, 0.125, 0.5, 0.0625),
+    ("ragged64_b32", 1, 2, 64, 333, 97, 32, 0.3, 0.5, 0.2),
+    ("no_pruning_all_sharp", 1, 2, 128, 256, 192, 64, 1.0, 0.0, 0.5),
+    ("all_flat_pooled_only", 1, 2, 128, 400, 300, 64, 0.5, 1.0, 0.0),
+    ("alpha_ns_one", 1, 2, 64, 256, 256, 64, 0.25, 0.5, 1.0),
+    ("single_ctx_block", 2, 2, 128, 512, 20, 64, 0.125, 0.5, 0.0625),
+    ("b32_d128", 1, 3, 128, 1024, 1024, 32, 0.125, 0.5, 0.0625),
+    ("odd_counts", 1, 1, 64, 700, 650, 64, 0.2, 0.37, 0.11),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_forward_small_cases(isa, case):
+    name, B, H, D, Ls, Lc, b, a_s, a_f, a_ns = case
+    check_case(isa, Workload(name, B, H, D, Ls, Lc, block=b, alpha_s=a_s, alpha_f=a_f, alpha_ns=a_ns, seed=31))
+
+
+def test_no_pruning_equals_dense(isa):
+    """alpha_s = 1, alpha_f = 0 reduces ISA to dense attention: the two CUDA
+    paths must agree with each other as well as with the oracle."""
+    w = Workload("np", 1, 2, 128, 384, 256, alpha_s=1.0, alpha_f=0.0, seed=9)
+    bits, out, _, _ = run_isa(isa, w)
+    q, k, v = (to_torch_bf16(x) for x in bits)
+    d = isa.dense(q, k, v, params_of(isa, w)).float().cpu().numpy().reshape(w.BH, w.L, w.D)
+    assert np.abs(d - out).max() <= 1e-2
+
+
+def test_forward_is_deterministic(isa):
+    w = Workload("det", 1, 2, 128, 512, 512, seed=3)
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    ws = isa.plan(q, k, v, p)
+    a = isa.forward(q, k, v, ws, p).clone()
+    b = isa.forward(q, k, v, ws, p)
+    ws2 = isa.plan(q, k, v, p)
+    c = isa.forward(q, k, v, ws2, p)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(a, c)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled
+# ---------------------------------------------------------------------------
+
+def test_forward_mid_full_size(isa):
+    """23768 tokens, H=8, D=128 (partial last block of each segment)."""
+    check_case(isa, named_workloads()["mid"], heads=range(8), blocks_per_head=10)
+
+
+def test_forward_dit14b_full_size(isa):
+    """The benchmarked workload: B=2, H=40, 16384 + 16384 tokens, D=128."""
+    w = named_workloads()["dit14b"]
+    heads = sorted({bh for bh, _ in sample_blocks(w, 5, 1)})
+    check_case(isa, w, heads=heads, blocks_per_head=6)
+
+
+# ---------------------------------------------------------------------------
+# bounded waits
+# ---------------------------------------------------------------------------
+
+def test_timeout_path_reports_status_and_context_survives(isa):
+    """Fault injection makes the attention kernel wait on a barrier nothing
+    arrives on; the wait must run out, raise the status word and return, and
+    the next normal launch must still be correct."""
+    w = Workload("to", 1, 1, 64, 128, 128, kind="iid", seed=1)
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    isa.set_wait_timeout_ns(2_000_000)
+    isa.set_fault_injection(1)
+    try:
+        isa.dense(q, k, v, p, status=status)
+        torch.cuda.synchronize()
+    finally:
+        isa.set_fault_injection(0)
+        isa.set_wait_timeout_ns(0)
+    assert int(status.item()) == isa.ISA_ERR_DEVICE_TIMEOUT
+    out = isa.dense(q, k, v, p, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, _ = O.dense_attention(*(bf16_to_f64(x.reshape(w.L, w.D)) for x in (qb, kb, vb)), 1 / 8.0)
+    assert np.abs(out.float().cpu().numpy().reshape(w.L, w.D) - ref).max() <= OUT_MAX_ABS
