@@ -1,0 +1,377 @@
+"""Benchmark of the ISA forward pass (isa_plan + isa_forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+One step = the whole hot path over one batch of synthetic input: pooling,
+coarse scores, context TopK, sharpness split, exact lists (isa_plan) and the
+fused sharp + flat attention (isa_forward).  Default workload: the 14B
+DiT-layer shape, B=2 (a CFG pair), H=40, D=128, 16384 source + 16384 context
+tokens, b=64, alpha_s=0.125, alpha_f=0.5, alpha_ns=0.0625, seeded clustered
+bf16 inputs (the pages' video latents are not available).
+
+Prints one JSON line.  `value` is executed TFLOP/s over all ranks (4*D per
+query-token x key-column pair, pooled blocks one column each, plus 2*T*T*D
+per head for the coarse scores), `latency_ms` the per-step latency.  With
+N > 1 (torchrun) every rank runs its own copy of the workload (heads are
+independent; no data-path collective), timing is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import Workload, generate_bits, named_workloads  # noqa: E402
+
+METRIC = "ISA fwd latency (ms) & executed TFLOP/s vs roofline at 32K/131K tokens, D=128"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def describe(w: Workload) -> dict:
+    return {"workload": f"{w.name}: B={w.B} H={w.H} D={w.D} L_src={w.L_src} L_ctx={w.L_ctx} b={w.block} "
+                        f"alpha_s={w.alpha_s} alpha_f={w.alpha_f} alpha_ns={w.alpha_ns}, {w.kind} bf16 seed {w.seed}",
+            "B": w.B, "H": w.H, "D": w.D, "L_src": w.L_src, "L_ctx": w.L_ctx, "block": w.block,
+            "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "alpha_ns": w.alpha_ns}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w: Workload, heads=(0, 1), per_kind=40, seed=11):
+    """Times the fp64 oracle on a bounded sample of the workload: the full
+    plan of `heads` plus `per_kind` sharp and `per_kind` flat query blocks of
+    each.  Returns (executed flops of the sample, seconds, description)."""
+    import oracle as O
+    from workloads import bf16_to_f64
+    p = O.Params(D=w.D, L_src=w.L_src, L_ctx=w.L_ctx, block=w.block, alpha_s=w.alpha_s, alpha_f=w.alpha_f,
+                 alpha_ns=w.alpha_ns)
+    qb, kb, vb = generate_bits(w, heads=list(heads))
+    flops = 0.0
+    secs = 0.0
+    for i, h in enumerate(heads):
+        q, k, v = bf16_to_f64(qb[i]), bf16_to_f64(kb[i]), bf16_to_f64(vb[i])
+        t0 = time.perf_counter()
+        pl = O.plan_head(q, k, v, p)
+        g = np.random.default_rng(seed + h)
+        sb = g.choice(pl.sharp, size=min(per_kind, len(pl.sharp)), replace=False) if len(pl.sharp) else []
+        fb = g.choice(pl.flat, size=min(per_kind, len(pl.flat)), replace=False) if len(pl.flat) else []
+        O.forward_head(q, k, v, pl, p, blocks=list(sb) + list(fb))
+        secs += time.perf_counter() - t0
+        cnt = pl.counts.astype(np.float64)
+        kv_tok = cnt[pl.kept].sum()
+        flops += 2.0 * pl.T * pl.T * w.D
+        flops += 4.0 * w.D * sum(cnt[b] * kv_tok for b in sb)
+        fpos = {int(b): r for r, b in enumerate(pl.flat)}
+        n_ex = pl.exact.shape[1]
+        for b in fb:
+            ex_tok = cnt[pl.kept[pl.exact[fpos[int(b)]]]].sum()
+            flops += 4.0 * w.D * cnt[b] * (ex_tok + len(pl.kept) - n_ex)
+    desc = (f"fp64 numpy oracle: full plan of heads {list(heads)} + {per_kind} sharp and {per_kind} flat "
+            f"query blocks of each, of {w.name}; rate scales to the whole workload")
+    return flops, secs, desc
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, w: Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    times, flops_total = [], 0.0
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        fl, secs, desc = oracle_sample(w, heads=(i % w.BH,), per_kind=8)
+        if i >= args.warmup:
+            times.append(secs)
+            flops_total += fl
+    sec = sum(times)
+    value = flops_total / sec / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": desc + "; one head and 8+8 blocks per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        load = [s for s, p in zip(sm, pw) if p is not None and p > 300] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_gpu(args, w: Workload):
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_coarse_b200 as isa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs: one full copy of the workload per rank, resident in HBM
+    wr = w.replace(seed=w.seed + 100 * rank) if world > 1 else w
+    qb, kb, vb = generate_bits(wr)
+
+    def to_dev(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+    ws = isa.alloc_workspace(p, dev)
+    out = torch.empty_like(q)
+
+    def step():
+        isa.plan(q, k, v, p, ws)
+        isa.forward(q, k, v, ws, p, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    view = isa.plan_view(p, ws)
+    status = int(view["status"].item())
+    flops = isa.executed_flops(p, view)
+    plan_flops = 2.0 * view["T"] ** 2 * w.D * w.BH
+    attn_flops = flops - plan_flops
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            isa.plan(q, k, v, p, ws)
+            ev[i][1].record(stream)
+            isa.forward(q, k, v, ws, p, out=out)
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    plan_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    fwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+
+    # the dense kernel on the same inputs
+    dense_ms = None
+    if not args.skip_dense:
+        for _ in range(2):
+            isa.dense(q, k, v, p, out=out)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = 3
+        e0.record(stream)
+        for _ in range(nd):
+            isa.dense(q, k, v, p, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms = e0.elapsed_time(e1) / nd
+
+    # end to end through the public API from pinned host memory
+    e2e = None
+    if not args.skip_e2e:
+        qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb))
+        for _ in range(2):
+            isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev)
+        torch.cuda.synchronize(dev)
+        ke = max(2, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ke):
+            res = isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / ke
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(3 * q.numel() * 2), "d2h_bytes_per_step": int(res.numel() * 2),
+               "ms_per_step": e2e_ms}
+        del qh, kh, vh, res
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    fwd_avg = statistics.mean(fwd_ms)
+    plan_avg = statistics.mean(plan_ms)
+    achieved = attn_flops / (fwd_avg / 1e3) / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    T = int(view["T"])
+    plan_bytes = 3 * q.numel() * 2 + 3 * w.BH * T * w.D * 4
+    traffic = None
+    tf_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tf_path):
+        try:
+            with open(tf_path) as f:
+                traffic = json.load(f).get(f"attn:{w.name}")
+        except (OSError, ValueError):
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "latency_ms": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded clustered generator, no trained weights)",
+        "config": {**describe(w), "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs {3 * q.numel() * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush)"},
+        "plan_ms": plan_avg, "forward_ms": fwd_avg, "executed_tflop_per_step": flops / 1e12,
+        "tflops_frac_sustained": achieved / peak_sus, "tflops_frac_burst": achieved / peak_burst,
+        "plan_hbm_gbs": plan_bytes / (plan_avg / 1e3) / 1e9,
+        "dense_ms": dense_ms, "speedup_vs_dense": (dense_ms / ms_per_step) if dense_ms else None,
+        "roofline": {"kernel": "attn_kernel (isa_forward)", "bound": "tensor", "achieved": achieved,
+                     "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                     "peak_kind": f"bf16 sustained ({peak_src})"},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and not args.skip_cpu:
+        fl, secs, desc = oracle_sample(w)
+        line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                "kind": "oracle", "sample": desc, "seconds": secs}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="dit14b")
+    ap.add_argument("--skip-dense", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    w = named_workloads()[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -119,6 +119,52 @@ __device__ __forceinline__ int3 kv_span(const AttnArgs& a, const Item& I, int j,
   return make_int3(r0, max(0, min(R, a.T_kv - r0)), 1);
 }
 
+// Column validity of one KV tile for one query row: bit c of mw[c/32] set
+// when column c takes part.  `masked` is warp-uniform (a row-independent
+// mask for sharp and dense tiles; flat tiles are always masked).
+struct TileMeta {
+  uint32_t mw[4];
+  int pooled, masked;
+};
+
+template <int R, int G>
+__device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, int j, int g_r,
+                                              const uint32_t* rbits) {
+  TileMeta m;
+  if (I.kind == 2 && j >= a.n_exact) {
+    // pooled tile: kept blocks [jp*128, jp*128+128) minus this row's exact blocks
+    const int jp = j - a.n_exact;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int rem = a.T_kv - (jp * 128 + 32 * w);
+      const uint32_t range = rem >= 32 ? 0xFFFFFFFFu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
+      const int wi = jp * 4 + w;
+      const uint32_t ex = rbits ? (wi < a.words ? rbits[wi] : 0u) : 0xFFFFFFFFu;
+      m.mw[w] = range & ~ex;
+    }
+    m.pooled = 1;
+    m.masked = 1;
+    return m;
+  }
+  int cnt[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) cnt[g] = kv_span<R, G>(a, I, j, g).y;
+  if (I.kind == 2) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) cnt[g] = (g == g_r) ? cnt[g] : 0;   // block-diagonal exact tiles
+  }
+  bool full = true;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int c = cnt[(w * 32) / R] - (w * 32) % R;
+    m.mw[w] = c >= 32 ? 0xFFFFFFFFu : (c <= 0 ? 0u : ((1u << c) - 1u));
+    full = full && m.mw[w] == 0xFFFFFFFFu;
+  }
+  m.pooled = 0;
+  m.masked = (I.kind == 2) ? 1 : (full ? 0 : 1);
+  return m;
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -128,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int G = C::G;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kNS], k_empty[kNS], v_full[kNS], v_empty[kNS];
-  __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done, o_free, drain_bar, inject_bar;
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done, o_ready, o_free, drain_bar, inject_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -150,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_empty[i], 1);
     }
     mbar_init(&pv_done, 1);
+    mbar_init(&o_ready, 1);
     mbar_init(&o_free, 128);
     mbar_init(&drain_bar, 1);
     mbar_init(&inject_bar, 1);
@@ -280,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       --t;   // the loop ran one step past the last tile
       tc_commit(&q_empty[qb]);
+      tc_commit(&o_ready);   // once per item: every P.V of the item landed in O
     }
     if (issued) {
       tc_commit(&drain_bar);
@@ -291,99 +339,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const int g_r = row / R, rr = row % R;
+    const float sl2 = a.sl2;
+    const float log2b = __log2f((float)a.b);
     int n = 0, t = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
       const Item I = decode_item<G>(a, it);
       const int2 qs = q_span<R>(a, I, g_r);
       const bool row_valid = rr < qs.y;
-      // pooled-tile data of this row's flat block
+      // pooled tiles of a flat item: this row's exact-block bitmap and the
+      // (at most two) partial kept blocks, whose weight is n_j instead of b
       const uint32_t* rbits = nullptr;
       int pb0 = -1, pb1 = -1;
-      float lb0 = 0.f, lb1 = 0.f;
-      const float log2b = __log2f((float)a.b);
+      float d0 = 0.f, d1 = 0.f;
       if (I.kind == 2) {
         const int f = I.slot0 + g_r;
         if (f < a.n_flat) rbits = a.bits + ((size_t)I.bh * a.n_flat + f) * a.words;
         if (a.L_src % a.b) {
           pb0 = a.T_src - 1;
-          lb0 = __log2f((float)(a.L_src % a.b));
+          d0 = (__log2f((float)(a.L_src % a.b)) - log2b) / sl2;
         }
         if ((a.L_ctx % a.b) && a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1) {
           pb1 = a.T_kv - 1;
-          lb1 = __log2f((float)(a.L_ctx % a.b));
+          d1 = (__log2f((float)(a.L_ctx % a.b)) - log2b) / sl2;
         }
       }
       float m_run = -INFINITY, l_run = 0.f;
+      TileMeta nxt = tile_meta<R, G>(a, I, 0, g_r, rbits);
       for (int j = 0; j < I.ntiles; ++j, ++t) {
+        const TileMeta cur = nxt;
+        if (j + 1 < I.ntiles) nxt = tile_meta<R, G>(a, I, j + 1, g_r, rbits);   // loads overlap the wait
         const int buf = t & 1;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t >> 1) & 1, wc))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(trow + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(trow + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(trow + buf * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(trow + buf * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        // column validity of this tile for this row
-        int cnt[G];
-        bool pooled = false;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const int3 sp = kv_span<R, G>(a, I, j, g);
-          cnt[g] = sp.y;
-          pooled = sp.z != 0;
-        }
-        if (I.kind == 2 && !pooled) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) cnt[g] = (g == g_r) ? cnt[g] : 0;   // block-diagonal
-        }
+        uint32_t sr[4][32];
+        tmem_ld32(trow + buf * 128 + 0, sr[0]);
+        tmem_ld32(trow + buf * 128 + 32, sr[1]);
+        tmem_ld32(trow + buf * 128 + 64, sr[2]);
+        tmem_ld32(trow + buf * 128 + 96, sr[3]);
         tmem_wait_ld();
-        float x[128];
-        if (pooled) {
-          const int jp = j - a.n_exact;
-          uint32_t wd[4];
+        float s[128];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int wi = jp * 4 + w;
-            wd[w] = (rbits && wi < a.words) ? rbits[wi] : 0xFFFFFFFFu;
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        if (cur.masked) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = ((cur.mw[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+          if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
+            const int kk0 = (j - a.n_exact) * 128;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
           }
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int kk = jp * 128 + c;
-            const bool valid = kk < a.T_kv && !((wd[c >> 5] >> (c & 31)) & 1u);
-            const float bias = kk == pb0 ? lb0 : (kk == pb1 ? lb1 : log2b);
-            x[c] = valid ? fmaf(__uint_as_float(sr[c]), a.sl2, bias) : -INFINITY;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            x[c] = ((c % R) < cnt[c / R]) ? __uint_as_float(sr[c]) * a.sl2 : -INFINITY;
         }
-        float mx = -INFINITY;
+        // row maximum of the tile: 8 independent chains of 3-input max
+        float mxa[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        for (int e = 0; e < 8; ++e) mxa[e] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
+        const float bias = cur.pooled ? log2b : 0.f;
+        const float mx =
+            fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])) * sl2 + bias;
         const bool need = mx > m_run + kRescaleLog2;
         const float m_new = need ? mx : m_run;
         const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
         const float alpha = need ? ex2(m_run - m_ref) : 1.f;
-        float sum = 0.f;
-        uint32_t pk[64];
+        const float neg = bias - m_ref;
+        // p = 2^(s * scale*log2e + bias - m_ref) in pairs; bf16 P for the MMA
+        float2 acc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+        uint32_t pk[2][32];
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2(x[c] - m_ref), p1 = ex2(x[c + 1] - m_ref);
-          sum += p0 + p1;
-          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-          pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h);
+          const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
+          const float p0 = ex2(x.x), p1 = ex2(x.y);
+          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(p0, p1));
+          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
         }
-        l_run = l_run * alpha + sum;
+        const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+        const float2 a03 = fadd2(a01, a23);
+        l_run = l_run * alpha + (a03.x + a03.y);
         m_run = m_new;
-        tmem_st32(trow + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(trow + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_st32(trow + buf * 128 + 0, pk[0]);
+        tmem_st32(trow + buf * 128 + 32, pk[1]);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
-          // rescale the running output once P.V of the previous tile landed
+          // rescale the running output once P.V of the previous tile landed.
+          // S_t (ready here) was issued after P.V of tile t-2, so pv_done has
+          // completed t-1 or t phases and the parity test is exact.
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) {
             ok = false;
             break;
@@ -404,12 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&p_full[buf]);
       }
       if (!ok) break;
-      // epilogue: wait for the last P.V, normalise, write rows in token order
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) break;
+      // epilogue: wait until every P.V of the item landed (a per-item barrier:
+      // pv_done may still be two phases behind here, because the last tile's
+      // S MMA was issued before the second-to-last P.V), normalise, write
+      // rows in token order
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_ready, n & 1, wc))) break;
       tc_fence_after();
-      uint32_t o[D];
+      uint32_t o[D / 32][32];
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(trow + 256 + c0, *reinterpret_cast<uint32_t(*)[32]>(&o[c0]));
+      for (int c0 = 0; c0 < D / 32; ++c0) tmem_ld32(trow + 256 + 32 * c0, o[c0]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&o_free);
@@ -420,14 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D; c += 8) {
           uint4 w;
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
-          w.x = *reinterpret_cast<uint32_t*>(&h0);
-          w.y = *reinterpret_cast<uint32_t*>(&h1);
-          w.z = *reinterpret_cast<uint32_t*>(&h2);
-          w.w = *reinterpret_cast<uint32_t*>(&h3);
+          const uint32_t* oc = &o[c >> 5][c & 31];
+          w.x = pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
           dst[c / 8] = w;
         }
         if (a.lse) {
