@@ -18,10 +18,12 @@
 // All tiles of an item update one online-softmax state per query row, so the
 // exact and the pooled terms share one normaliser.
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0 lane 0 : TMA producer (Q tile double-buffered, K/V in kNS stages)
+// Roles (352 threads, one CTA per SM):
+//   warp 0 lane 0 : TMA producer of the Q tile and the K tiles (kNSK stages)
 //   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma
-//   warps 2..5    : softmax / correction / epilogue, thread = query row
+//   warps 2..9    : softmax / correction / epilogue; each query row is
+//                   handled by two threads (64 columns of the S tile each)
+//   warp 10 lane 0: TMA producer of the V tiles (kNSV stages)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O [256, 256+D).  P (bf16)
 // overwrites the first 64 columns of its S buffer and feeds the P.V MMA as the
 // A operand straight from TMEM.
@@ -29,9 +31,13 @@
 
 namespace isa {
 
-constexpr int kThreads = 192;
-constexpr int kNS = 2;              // K/V pipeline stages
+constexpr int kThreads = 352;      // 11 warps: Q/K producer, MMA, 8 softmax, V producer
+constexpr int kNSK = 3;             // K pipeline stages
+constexpr int kNSV = 2;             // V pipeline stages
 constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
+// Exponentials of column pairs p with bit (p % 8) set go through the cubic on
+// the FMA pipe, the rest through MUFU: 3 of 8 balances the two pipes.
+constexpr uint32_t kPolyPairs = 0x11u;
 
 template <int D, int R>
 struct Cfg {
@@ -40,12 +46,12 @@ struct Cfg {
   static constexpr uint32_t CHUNK = 128 * 128;             // 128 rows x 128 bytes
   static constexpr uint32_t TILE = 128 * D * 2;            // one 128-row tile
   static constexpr uint32_t BOX = R * 128;                 // one TMA box
-  static constexpr uint32_t Q_OFF = 0;                     // 2 buffers
-  static constexpr uint32_t K_OFF = 2 * TILE;
-  static constexpr uint32_t V_OFF = K_OFF + kNS * TILE;
+  static constexpr uint32_t Q_OFF = 0;                     // one Q tile
+  static constexpr uint32_t K_OFF = TILE;
+  static constexpr uint32_t V_OFF = K_OFF + kNSK * TILE;
   // + 1024 alignment slack; at least 120 KB so that only one CTA (and one
   // 512-column TMEM allocation) fits on an SM
-  static constexpr uint32_t SMEM_USED = V_OFF + kNS * TILE + 1024;
+  static constexpr uint32_t SMEM_USED = V_OFF + kNSV * TILE + 1024;
   static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0);
   static constexpr uint32_t ID_O = idesc_bf16_f32(128, D, 1);
@@ -119,6 +125,21 @@ __device__ __forceinline__ int3 kv_span(const AttnArgs& a, const Item& I, int j,
   return make_int3(r0, max(0, min(R, a.T_kv - r0)), 1);
 }
 
+// Per-item constants that give the valid-token count of any kept block
+// without a memory access: only the last source block and the last context
+// block can be partial, and the latter is kept only as the last kept block.
+struct ItemCounts {
+  int src_tail;     // tokens of block T_src-1
+  int kv_tail;      // tokens of kept block T_kv-1
+};
+
+__device__ __forceinline__ int kept_count(const AttnArgs& a, const ItemCounts& ic, int kk) {
+  if (kk >= a.T_kv || kk < 0) return 0;
+  if (kk == a.T_src - 1) return ic.src_tail;
+  if (kk == a.T_kv - 1) return ic.kv_tail;
+  return a.b;
+}
+
 // Column validity of one KV tile for one query row: bit c of mw[c/32] set
 // when column c takes part.  `masked` is warp-uniform (a row-independent
 // mask for sharp and dense tiles; flat tiles are always masked).
@@ -127,9 +148,21 @@ struct TileMeta {
   int pooled, masked;
 };
 
+// exact-block positions (in the kept list) of the G query blocks of a flat
+// item for exact tile j: loaded one tile ahead of their use
+template <int G>
+__device__ __forceinline__ void load_exact(const AttnArgs& a, const Item& I, int j, int (&kk)[G]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int f = I.slot0 + g;
+    kk[g] = (I.kind == 2 && j < a.n_exact && f < a.n_flat) ? a.exact[((size_t)I.bh * a.n_flat + f) * a.n_exact + j]
+                                                             : -1;
+  }
+}
+
 template <int R, int G>
-__device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, int j, int g_r,
-                                              const uint32_t* rbits) {
+__device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, const ItemCounts& ic, int j, int g_r,
+                                              const uint32_t* rbits, const int (&ekk)[G]) {
   TileMeta m;
   if (I.kind == 2 && j >= a.n_exact) {
     // pooled tile: kept blocks [jp*128, jp*128+128) minus this row's exact blocks
@@ -148,10 +181,15 @@ __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, 
   }
   int cnt[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g) cnt[g] = kv_span<R, G>(a, I, j, g).y;
-  if (I.kind == 2) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) cnt[g] = (g == g_r) ? cnt[g] : 0;   // block-diagonal exact tiles
+  for (int g = 0; g < G; ++g) {
+    if (I.kind == 0) {
+      const int s0 = j * 128 + g * R;
+      cnt[g] = max(0, min(R, a.L - s0));
+    } else if (I.kind == 1) {
+      cnt[g] = kept_count(a, ic, j * G + g);
+    } else {
+      cnt[g] = (g == g_r) ? kept_count(a, ic, ekk[g]) : 0;   // block-diagonal exact tiles
+    }
   }
   bool full = true;
 #pragma unroll
@@ -173,8 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<D, R>;
   constexpr int G = C::G;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kNS], k_empty[kNS], v_full[kNS], v_empty[kNS];
+  __shared__ __align__(8) uint64_t q_full, q_empty, k_full[kNSK], k_empty[kNSK], v_full[kNSV], v_empty[kNSV];
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done, o_ready, o_free, drain_bar, inject_bar;
+  __shared__ __align__(8) uint64_t pair_max[4], pair_sum[4];   // the two softmax warps of one lane quarter
+  __shared__ float xmax[2][128][2];   // per tile parity, row, half: raw row maximum of the half
+  __shared__ float xsum[128][2];      // per row, half: softmax normaliser of the half
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -183,21 +224,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
 
   if (tid == 0) {
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
     }
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < kNSK; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kNSV; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
     mbar_init(&pv_done, 1);
     mbar_init(&o_ready, 1);
-    mbar_init(&o_free, 128);
+    mbar_init(&o_free, 256);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&pair_max[i], 64);
+      mbar_init(&pair_sum[i], 64);
+    }
     mbar_init(&drain_bar, 1);
     mbar_init(&inject_bar, 1);
     abort_flag = 0;
@@ -217,27 +264,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   const WaitCtl wc{&abort_flag, a.status, a.timeout_ns};
 
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    int q_cnt[2] = {0, 0}, k_cnt[kNS], v_cnt[kNS];
-    for (int i = 0; i < kNS; ++i) k_cnt[i] = v_cnt[i] = 0;
+  if ((warp == 0 || warp == 10) && lane == 0) {
+    // ------------------------------------------------------------ producers
+    // warp 0: Q tile and K tiles; warp 10: V tiles.  Separate threads keep
+    // the K stream kNSK tiles and the V stream kNSV tiles ahead of the MMA
+    // independently of each other.
+    const bool kside = warp == 0;
+    int q_cnt = 0, cnt[kNSK > kNSV ? kNSK : kNSV];
+    const int ns = kside ? kNSK : kNSV;
+    for (int i = 0; i < ns; ++i) cnt[i] = 0;
+    uint64_t* full = kside ? k_full : v_full;
+    uint64_t* empty = kside ? k_empty : v_empty;
+    const uint32_t off = kside ? C::K_OFF : C::V_OFF;
     int n = 0, t = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
       const Item I = decode_item<G>(a, it);
-      const int qb = n & 1;
-      if (n >= 2 && !mbar_wait(&q_empty[qb], ((n >> 1) - 1) & 1, wc)) break;
-      mbar_arrive_expect_tx(&q_full[qb], C::TILE);
-      ++q_cnt[qb];
-      for (int g = 0; g < G; ++g) {
-        const int2 sp = q_span<R>(a, I, g);
-        const int row = I.bh * a.L + (sp.y > 0 ? sp.x : 0);
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_2d(sgen + C::Q_OFF + qb * C::TILE + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[qb]);
+      if (kside) {
+        if (n >= 1 && !mbar_wait(&q_empty, (n - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&q_full, C::TILE);
+        ++q_cnt;
+        for (int g = 0; g < G; ++g) {
+          const int2 sp = q_span<R>(a, I, g);
+          const int row = I.bh * a.L + (sp.y > 0 ? sp.x : 0);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_2d(sgen + C::Q_OFF + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full);
+        }
       }
       for (int j = 0; j < I.ntiles; ++j, ++t) {
-        const int s = t % kNS;
-        if (t >= kNS && !mbar_wait(&k_empty[s], ((t / kNS) - 1) & 1, wc)) {
+        const int s = t % ns;
+        if (t >= ns && !mbar_wait(&empty[s], ((t / ns) - 1) & 1, wc)) {
           ok = false;
           break;
         }
@@ -248,48 +304,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           pooled = sp.z != 0;
           rows[g] = pooled ? I.bh * a.T_kv_pad + sp.x : I.bh * a.L + (sp.y > 0 ? sp.x : 0);
         }
-        const CUtensorMap* mk = pooled ? &tm_kp : &tm_k;
-        const CUtensorMap* mv = pooled ? &tm_vp : &tm_v;
-        mbar_arrive_expect_tx(&k_full[s], C::TILE);
-        ++k_cnt[s];
+        const CUtensorMap* m = kside ? (pooled ? &tm_kp : &tm_k) : (pooled ? &tm_vp : &tm_v);
+        mbar_arrive_expect_tx(&full[s], C::TILE);
+        ++cnt[s];
         for (int g = 0; g < G; ++g)
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_2d(sgen + C::K_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, mk, c * 64, rows[g], &k_full[s]);
-        if (t >= kNS && !mbar_wait(&v_empty[s], ((t / kNS) - 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[s], C::TILE);
-        ++v_cnt[s];
-        for (int g = 0; g < G; ++g)
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_2d(sgen + C::V_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, mv, c * 64, rows[g], &v_full[s]);
+            tma_load_2d(sgen + off + s * C::TILE + c * C::CHUNK + g * C::BOX, m, c * 64, rows[g], &full[s]);
       }
     }
     // let every copy in flight land before the CTA can exit
-    for (int i = 0; i < 2; ++i)
-      if (q_cnt[i]) mbar_wait_drain(&q_full[i], (q_cnt[i] - 1) & 1, a.timeout_ns);
-    for (int i = 0; i < kNS; ++i) {
-      if (k_cnt[i]) mbar_wait_drain(&k_full[i], (k_cnt[i] - 1) & 1, a.timeout_ns);
-      if (v_cnt[i]) mbar_wait_drain(&v_full[i], (v_cnt[i] - 1) & 1, a.timeout_ns);
-    }
+    if (q_cnt) mbar_wait_drain(&q_full, (q_cnt - 1) & 1, a.timeout_ns);
+    for (int i = 0; i < ns; ++i)
+      if (cnt[i]) mbar_wait_drain(&full[i], (cnt[i] - 1) & 1, a.timeout_ns);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     bool issued = false, ok = true;
     if (a.inject) ok = mbar_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
     int n = 0, t = 0;
     const uint32_t tS = tmem, tO = tmem + 256;
+    const uint32_t qaddr = sbase + C::Q_OFF;
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
       const Item I = decode_item<G>(a, it);
-      const int qb = n & 1;
-      if (!mbar_wait(&q_full[qb], (n >> 1) & 1, wc)) break;
+      if (!mbar_wait(&q_full, n & 1, wc)) break;
       tc_fence_after();
-      const uint32_t qaddr = sbase + C::Q_OFF + qb * C::TILE;
       for (int j = 0; ok && j <= I.ntiles; ++j, ++t) {
         if (j < I.ntiles) {
           // S_t = Q K_t^T into S buffer t&1
-          const int s = t % kNS;
-          if (!mbar_wait(&k_full[s], (t / kNS) & 1, wc)) {
+          const int s = t % kNSK;
+          if (!mbar_wait(&k_full[s], (t / kNSK) & 1, wc)) {
             ok = false;
             break;
           }
@@ -297,19 +339,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-            mma_ss(tS + (t & 1) * 128, smem_desc_sw128(qaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024),
+            const uint32_t o = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+            mma_ss(tS + (t & 1) * 128, smem_desc_sw128(qaddr + o, 16, 1024), smem_desc_sw128(kaddr + o, 16, 1024),
                    C::ID_S, ks > 0);
           }
           issued = true;
           tc_commit(&s_full[t & 1]);
           tc_commit(&k_empty[s]);
+          if (j == I.ntiles - 1) tc_commit(&q_empty);   // last read of this item's Q
         }
         if (j > 0) {
           // O (+)= P_{t-1} V_{t-1}
-          const int tp = t - 1, sp = tp % kNS;
+          const int tp = t - 1, sp = tp % kNSV;
           const bool first = (j == 1);
-          if (!mbar_wait(&p_full[tp & 1], (tp >> 1) & 1, wc) || !mbar_wait(&v_full[sp], (tp / kNS) & 1, wc) ||
+          if (!mbar_wait(&p_full[tp & 1], (tp >> 1) & 1, wc) || !mbar_wait(&v_full[sp], (tp / kNSV) & 1, wc) ||
               (first && n > 0 && !mbar_wait(&o_free, (n - 1) & 1, wc))) {
             ok = false;
             break;
@@ -326,21 +369,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       --t;   // the loop ran one step past the last tile
-      tc_commit(&q_empty[qb]);
       tc_commit(&o_ready);   // once per item: every P.V of the item landed in O
     }
     if (issued) {
       tc_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, a.timeout_ns);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------ softmax
-    const int quarter = warp & 3;
+    // Warps 2..9.  Two warps share each TMEM lane quarter (tcgen05.ld reaches
+    // lanes 32*(warp%4)..+31): half h = 0 takes columns 0..63 of the S tile,
+    // h = 1 columns 64..127, of the same 32 query rows.  The halves agree on
+    // the row maximum every tile through shared memory, keep separate
+    // partial normalisers, and combine them in the epilogue.
+    const int quarter = warp & 3, h = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const int g_r = row / R, rr = row % R;
     const float sl2 = a.sl2;
     const float log2b = __log2f((float)a.b);
+    constexpr int DH = D / 2;           // output columns of this half
     int n = 0, t = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
@@ -364,44 +412,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           d1 = (__log2f((float)(a.L_ctx % a.b)) - log2b) / sl2;
         }
       }
+      ItemCounts ic;
+      ic.src_tail = a.L_src - (a.T_src - 1) * a.b;
+      ic.kv_tail = a.b;
+      if (I.kind != 0 && a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1)
+        ic.kv_tail = a.L_ctx - (a.T_ctx - 1) * a.b;
       float m_run = -INFINITY, l_run = 0.f;
-      TileMeta nxt = tile_meta<R, G>(a, I, 0, g_r, rbits);
+      int ekk[G];
+      load_exact<G>(a, I, 0, ekk);
       for (int j = 0; j < I.ntiles; ++j, ++t) {
-        const TileMeta cur = nxt;
-        if (j + 1 < I.ntiles) nxt = tile_meta<R, G>(a, I, j + 1, g_r, rbits);   // loads overlap the wait
+        const TileMeta cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
+        load_exact<G>(a, I, j + 1, ekk);   // next tile's indices; the loads overlap this tile
         const int buf = t & 1;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t >> 1) & 1, wc))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t sr[4][32];
-        tmem_ld32(trow + buf * 128 + 0, sr[0]);
-        tmem_ld32(trow + buf * 128 + 32, sr[1]);
-        tmem_ld32(trow + buf * 128 + 64, sr[2]);
-        tmem_ld32(trow + buf * 128 + 96, sr[3]);
+        uint32_t sr[2][32];
+        tmem_ld32(trow + buf * 128 + 64 * h, sr[0]);
+        tmem_ld32(trow + buf * 128 + 64 * h + 32, sr[1]);
         tmem_wait_ld();
-        float s[128];
+        float s[64];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
         if (cur.masked) {
+          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = ((cur.mw[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+          for (int c = 0; c < 64; ++c) s[c] = ((((c < 32) ? w0 : w1) >> (c & 31)) & 1u) ? s[c] : -INFINITY;
           if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
-            const int kk0 = (j - a.n_exact) * 128;
+            const int kk0 = (j - a.n_exact) * 128 + 64 * h;
 #pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
+            for (int c = 0; c < 64; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
           }
         }
-        // row maximum of the tile: 8 independent chains of 3-input max
+        // half-row maximum: 8 independent chains of 3-input max
         float mxa[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mxa[e] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
+        for (int c = 0; c < 64; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
+        const float mh = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+        xmax[buf][row][h] = mh;
+        mbar_arrive(&pair_max[quarter]);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pair_max[quarter], t & 1, wc))) {
+          ok = false;
+          break;
+        }
         const float bias = cur.pooled ? log2b : 0.f;
-        const float mx =
-            fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])) * sl2 + bias;
+        const float mx = fmaxf(mh, xmax[buf][row][h ^ 1]) * sl2 + bias;
         const bool need = mx > m_run + kRescaleLog2;
         const float m_new = need ? mx : m_run;
         const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
@@ -411,37 +470,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 acc[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
-        uint32_t pk[2][32];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
-          const float p0 = ex2(x.x), p1 = ex2(x.y);
-          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(p0, p1));
-          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
+          float2 pp;
+          if (kPolyPairs & (1u << ((c >> 1) & 7))) {
+            pp = ex2_poly2(x);             // FMA/ALU pipes
+          } else {
+            pp.x = ex2(x.x);               // MUFU
+            pp.y = ex2(x.y);
+          }
+          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pp);
+          pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
+        }
+        if (cur.masked) {
+          // the polynomial leaves masked columns at a denormal: clear them in P
+          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t bits = ((e < 16 ? w0 : w1) >> ((2 * e) & 31)) & 3u;
+            pk[e] &= (bits & 1u ? 0x0000FFFFu : 0u) | (bits & 2u ? 0xFFFF0000u : 0u);
+          }
         }
         const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const float2 a03 = fadd2(a01, a23);
         l_run = l_run * alpha + (a03.x + a03.y);
         m_run = m_new;
-        tmem_st32(trow + buf * 128 + 0, pk[0]);
-        tmem_st32(trow + buf * 128 + 32, pk[1]);
+        tmem_st32(trow + buf * 128 + 32 * h, pk);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
-          // rescale the running output once P.V of the previous tile landed.
-          // S_t (ready here) was issued after P.V of tile t-2, so pv_done has
-          // completed t-1 or t phases and the parity test is exact.
+          // rescale this half of the running output once P.V of the previous
+          // tile landed.  S_t (ready here) was issued after P.V of tile t-2,
+          // so pv_done has completed t-1 or t phases and the parity test is
+          // exact.
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = 0; c0 < DH; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(trow + 256 + c0, o);
+            tmem_ld32(trow + 256 + DH * h + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(trow + 256 + c0, o);
+            tmem_st32(trow + 256 + DH * h + c0, o);
           }
         }
         tmem_wait_st();
@@ -451,22 +525,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: wait until every P.V of the item landed (a per-item barrier:
       // pv_done may still be two phases behind here, because the last tile's
-      // S MMA was issued before the second-to-last P.V), normalise, write
-      // rows in token order
+      // S MMA was issued before the second-to-last P.V), combine the two
+      // halves' normalisers, normalise and write this half of each row
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_ready, n & 1, wc))) break;
       tc_fence_after();
-      uint32_t o[D / 32][32];
+      uint32_t o[DH / 32][32];
 #pragma unroll
-      for (int c0 = 0; c0 < D / 32; ++c0) tmem_ld32(trow + 256 + 32 * c0, o[c0]);
+      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld32(trow + 256 + DH * h + 32 * c0, o[c0]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&o_free);
+      xsum[row][h] = l_run;
+      mbar_arrive(&pair_sum[quarter]);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pair_sum[quarter], n & 1, wc))) break;
+      const float l_tot = l_run + xsum[row][h ^ 1];
       if (row_valid) {
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
-        uint4* dst = reinterpret_cast<uint4*>(a.out + tok * D);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + tok * D + DH * h);
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
+        for (int c = 0; c < DH; c += 8) {
           uint4 w;
           const uint32_t* oc = &o[c >> 5][c & 31];
           w.x = pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
@@ -475,9 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
           dst[c / 8] = w;
         }
-        if (a.lse) {
+        if (a.lse && h == 0) {
           const float mref = m_run == -INFINITY ? 0.f : m_run;
-          a.lse[tok] = (mref + __log2f(l_run)) * 0.69314718055994531f;
+          a.lse[tok] = (mref + __log2f(l_tot)) * 0.69314718055994531f;
         }
       }
     }
