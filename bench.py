@@ -50,6 +50,27 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def attn_traffic(workload: str):
+    """Measured DRAM bytes per attention launch (profiles/attn_traffic.txt), or
+    None when the kernel source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_attention_coarse_b200", "csrc", "isa_attn.cu")
+    try:
+        vals = {}
+        for line in open(path):
+            line = line.split("#", 1)[0].strip()
+            if "=" in line:
+                k, v = (x.strip() for x in line.split("=", 1))
+                vals[k] = v
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if vals.get("kernel_source_sha256") != sha or workload not in vals:
+        return None
+    return int(vals[workload])
+
+
 def describe(w: Workload) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.H} D={w.D} L_src={w.L_src} L_ctx={w.L_ctx} b={w.block} "
                         f"alpha_s={w.alpha_s} alpha_f={w.alpha_f} alpha_ns={w.alpha_ns}, {w.kind} bf16 seed {w.seed}",
@@ -61,7 +82,7 @@ def describe(w: Workload) -> dict:
 # CPU oracle timing (the reported baseline and the reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(w: Workload, heads=(0, 1), per_kind=40, seed=11):
+def oracle_sample(w: Workload, heads=(0, 1, 2, 3), per_kind=160, seed=11):
     """Times the fp64 oracle on a bounded sample of the workload: the full
     plan of `heads` plus `per_kind` sharp and `per_kind` flat query blocks of
     each.  Returns (executed flops of the sample, seconds, description)."""
@@ -152,10 +173,10 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.2)
         return self
 
     def __exit__(self, *exc):
@@ -320,14 +341,7 @@ def run_gpu(args, w: Workload):
     hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
     T = int(view["T"])
     plan_bytes = 3 * q.numel() * 2 + 3 * w.BH * T * w.D * 4
-    traffic = None
-    tf_path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tf_path):
-        try:
-            with open(tf_path) as f:
-                traffic = json.load(f).get(f"attn:{w.name}")
-        except (OSError, ValueError):
-            traffic = None
+    traffic = attn_traffic(w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "latency_ms": ms_per_step,
