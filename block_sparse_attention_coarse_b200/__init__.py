@@ -36,6 +36,7 @@ ISA_ERR_DEVICE_TIMEOUT = 5
 EXPORTS = (
     "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
+    "isa_forward_static",
 )
 
 
@@ -88,6 +89,8 @@ def load_library() -> ctypes.CDLL:
     lib.isa_version.restype = ctypes.c_char_p
     lib.isa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.isa_set_fault_injection.argtypes = [ctypes.c_int32]
+    lib.isa_forward_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.isa_forward_static.restype = ctypes.c_int
     for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
                  "isa_set_wait_timeout_ns", "isa_set_fault_injection"):
         getattr(lib, name).restype = ctypes.c_int

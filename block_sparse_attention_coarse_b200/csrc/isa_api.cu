@@ -180,6 +180,12 @@ int sm_count() {
 
 }  // namespace
 
+namespace isa {
+// Sets the calling thread's isa_last_error() text (used by other files of the
+// library that report their own errors).
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace isa
+
 extern "C" {
 
 isa_status isa_plan_workspace_size(const isa_params* p, size_t* bytes) {

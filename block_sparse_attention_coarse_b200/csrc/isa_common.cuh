@@ -59,6 +59,7 @@ cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void
                         cudaStream_t st);
 cudaError_t prepare_plan_kernels();
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
+void set_last_error(const char* msg);
 
 constexpr int kMaxT = 8192;      // blocks per head
 constexpr int kMaxTkv = 6144;    // kept blocks per head

@@ -138,6 +138,27 @@ isa_status isa_forward(const isa_params* p, const void* q, const void* k, const 
 isa_status isa_dense(const isa_params* p, const void* q, const void* k, const void* v,
                      void* out, float* lse, int32_t* status, void* stream);
 
+/* isa_plan + isa_forward for callers that cannot allocate device memory.
+ * The pages describe nothing like it (the paper has no counterpart): it
+ * serves callers that cannot hand the library a workspace -- code that must
+ * not call cudaMalloc (inside an allocator or memory-pool callback, a
+ * real-time loop that forbids allocation) or a binding without a device
+ * allocator.  The plan lives in a fixed 16 MiB device array inside the
+ * library; every GPU that loads the library holds it until the process
+ * exits.  Inputs, output and lse are as for isa_forward.
+ *  - A problem whose plan needs more than 16 MiB (isa_plan_workspace_size)
+ *    returns ISA_ERR_WORKSPACE with a message; nothing is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Allocates nothing (no cudaMalloc/cudaFree, no library allocation).
+ *  - All calls share the one array, which keeps the last call's contents;
+ *    every plan entry is rewritten and the status word cleared by each call.
+ *    Calls that overlap on the GPU race on the array: order them.
+ * Device timeouts are reported as for isa_forward, in the array's status
+ * word (not readable by the caller; use isa_plan/isa_forward to inspect). */
+isa_status isa_forward_static(const isa_params* p, const void* q, const void* k, const void* v, void* out,
+                              float* lse, void* stream);
+
 /* Thread-local description of the last error (never NULL). */
 const char* isa_last_error(void);
 
