@@ -20,11 +20,13 @@
 //
 // Roles (352 threads, one CTA per SM):
 //   warp 0 lane 0 : TMA producer of the Q tile and the K tiles (kNSK stages)
-//   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma
+//   warp 1        : allocates TMEM; runs the MMA loop as one converged warp,
+//                   one elected lane issuing each tcgen05.mma / commit
 //   warps 2..9    : softmax / correction / epilogue; each query row is
 //                   handled by two threads (64 columns of the S tile each)
 //   warp 10 lane 0: TMA producer of the V tiles (kNSV stages)
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256, 256+D).  P (bf16)
+// TMEM (512 columns): S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+D).
+// S of tile t lives in buffer t % 3, so S runs two tiles ahead of P.V.  P (bf16)
 // overwrites the first 64 columns of its S buffer and feeds the P.V MMA as the
 // A operand straight from TMEM.
 #include "isa_common.cuh"
@@ -35,8 +37,9 @@ constexpr int kThreads = 352;      // 11 warps: Q/K producer, MMA, 8 softmax, V 
 constexpr int kNSK = 3;             // K pipeline stages
 constexpr int kNSV = 2;             // V pipeline stages
 constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
+constexpr uint32_t kTmemO = 384;    // TMEM column of O (after three 128-column S buffers)
 // Exponentials of column pairs p with bit (p % 8) set go through the cubic on
-// the FMA pipe, the rest through MUFU: 3 of 8 balances the two pipes.
+// the FMA pipe, the rest through MUFU (2 of 8).
 constexpr uint32_t kPolyPairs = 0x11u;
 
 template <int D, int R>
@@ -203,6 +206,11 @@ __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, 
   return m;
 }
 
+// Warp-uniform bounded wait: every lane waits, the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, w));
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -212,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int G = C::G;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[kNSK], k_empty[kNSK], v_full[kNSV], v_empty[kNSV];
-  __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done, o_ready, o_free, drain_bar, inject_bar;
+  __shared__ __align__(8) uint64_t s_full[3], p_full[3], pv_done[2], o_ready, o_free, drain_bar, inject_bar;
   __shared__ __align__(8) uint64_t pair_max[4], pair_sum[4];   // the two softmax warps of one lane quarter
-  __shared__ float xmax[2][128][2];   // per tile parity, row, half: raw row maximum of the half
+  __shared__ float xmax[3][128][2];   // per S buffer, row, half: raw row maximum of the half
   __shared__ float xsum[128][2];      // per row, half: softmax normaliser of the half
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&q_full, 1);
     mbar_init(&q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 256);
     }
@@ -238,7 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    mbar_init(&pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(&o_ready, 1);
     mbar_init(&o_free, 256);
     for (int i = 0; i < 4; ++i) {
@@ -316,63 +325,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (q_cnt) mbar_wait_drain(&q_full, (q_cnt - 1) & 1, a.timeout_ns);
     for (int i = 0; i < ns; ++i)
       if (cnt[i]) mbar_wait_drain(&full[i], (cnt[i] - 1) & 1, a.timeout_ns);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop in lockstep, so every descriptor and TMEM
+    // address is warp-uniform; one elected lane issues each tcgen05 op.  S of
+    // tile t+2 is issued before P.V of tile t (three S buffers), so the
+    // softmax of the next two tiles never waits for the P.V round trip.
     bool issued = false, ok = true;
-    if (a.inject) ok = mbar_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
-    int n = 0, t = 0;
-    const uint32_t tS = tmem, tO = tmem + 256;
+    if (a.inject) ok = warp_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
+    int n = 0, t0 = 0;   // items so far, global index of the item's first tile
+    const uint32_t tO = tmem + kTmemO;
     const uint32_t qaddr = sbase + C::Q_OFF;
+    // S_t = Q K_t^T into S buffer t % 3
+    auto issue_s = [&](int t, bool last) -> bool {
+      const int s = t % kNSK;
+      if (!warp_wait(&k_full[s], (t / kNSK) & 1, wc)) return false;
+      tc_fence_after();
+      const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
+      const uint32_t tS = tmem + (t % 3) * 128;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+        mma_ss_elect(tS, smem_desc_sw128(qaddr + o, 16, 1024), smem_desc_sw128(kaddr + o, 16, 1024), C::ID_S, ks > 0);
+      }
+      issued = true;
+      tc_commit_elect(&s_full[t % 3]);
+      tc_commit_elect(&k_empty[s]);
+      if (last) tc_commit_elect(&q_empty);   // last read of this item's Q
+      return true;
+    };
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
       const Item I = decode_item<G>(a, it);
-      if (!mbar_wait(&q_full, n & 1, wc)) break;
+      const int nt = I.ntiles;
+      if (!warp_wait(&q_full, n & 1, wc)) break;
       tc_fence_after();
-      for (int j = 0; ok && j <= I.ntiles; ++j, ++t) {
-        if (j < I.ntiles) {
-          // S_t = Q K_t^T into S buffer t&1
-          const int s = t % kNSK;
-          if (!mbar_wait(&k_full[s], (t / kNSK) & 1, wc)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t o = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-            mma_ss(tS + (t & 1) * 128, smem_desc_sw128(qaddr + o, 16, 1024), smem_desc_sw128(kaddr + o, 16, 1024),
-                   C::ID_S, ks > 0);
-          }
-          issued = true;
-          tc_commit(&s_full[t & 1]);
-          tc_commit(&k_empty[s]);
-          if (j == I.ntiles - 1) tc_commit(&q_empty);   // last read of this item's Q
+      for (int j = 0; ok && j < nt && j < 2; ++j) ok = issue_s(t0 + j, j == nt - 1);
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 2 < nt && !(ok = issue_s(t0 + j + 2, j + 2 == nt - 1))) break;
+        // O (+)= P_tp V_tp
+        const int tp = t0 + j, sp = tp % kNSV, pb = tp % 3;
+        if (!warp_wait(&p_full[pb], (tp / 3) & 1, wc) || !warp_wait(&v_full[sp], (tp / kNSV) & 1, wc) ||
+            (j == 0 && n > 0 && !warp_wait(&o_free, (n - 1) & 1, wc))) {
+          ok = false;
+          break;
         }
-        if (j > 0) {
-          // O (+)= P_{t-1} V_{t-1}
-          const int tp = t - 1, sp = tp % kNSV;
-          const bool first = (j == 1);
-          if (!mbar_wait(&p_full[tp & 1], (tp >> 1) & 1, wc) || !mbar_wait(&v_full[sp], (tp / kNSV) & 1, wc) ||
-              (first && n > 0 && !mbar_wait(&o_free, (n - 1) & 1, wc))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t vaddr = sbase + C::V_OFF + sp * C::TILE;
+        tc_fence_after();
+        const uint32_t vaddr = sbase + C::V_OFF + sp * C::TILE;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ts(tO, tS + (tp & 1) * 128 + ks * 8, smem_desc_sw128(vaddr + ks * 2048, C::CHUNK, 1024), C::ID_O,
-                   (!first || ks > 0) ? 1u : 0u);
-          tc_commit(&v_empty[sp]);
-          tc_commit(&pv_done);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_elect(tO, tmem + pb * 128 + ks * 8, smem_desc_sw128(vaddr + ks * 2048, C::CHUNK, 1024), C::ID_O,
+                       (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit_elect(&v_empty[sp]);
+        tc_commit_elect(&pv_done[tp & 1]);
       }
       if (!ok) break;
-      --t;   // the loop ran one step past the last tile
-      tc_commit(&o_ready);   // once per item: every P.V of the item landed in O
+      tc_commit_elect(&o_ready);   // once per item: every P.V of the item landed in O
+      t0 += nt;
     }
     if (issued) {
-      tc_commit(&drain_bar);
+      tc_commit_elect(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, a.timeout_ns);
     }
   } else if (warp >= 2 && warp <= 9) {
@@ -418,13 +429,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (I.kind != 0 && a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1)
         ic.kv_tail = a.L_ctx - (a.T_ctx - 1) * a.b;
       float m_run = -INFINITY, l_run = 0.f;
+      int jm0 = -1, jm1 = -1;
+      if (I.kind == 1) {
+        if (ic.src_tail != a.b) jm0 = (a.T_src - 1) / G;
+        jm1 = (a.T_kv - 1) / G;
+      } else if (I.kind == 0) {
+        jm1 = (a.L - 1) / 128;
+      }
       int ekk[G];
       load_exact<G>(a, I, 0, ekk);
       for (int j = 0; j < I.ntiles; ++j, ++t) {
-        const TileMeta cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
-        load_exact<G>(a, I, j + 1, ekk);   // next tile's indices; the loads overlap this tile
-        const int buf = t & 1;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t >> 1) & 1, wc))) {
+        TileMeta cur;
+        if (I.kind == 2 || j == jm0 || j == jm1) {
+          cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
+          load_exact<G>(a, I, j + 1, ekk);
+        } else {
+          cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
+          cur.pooled = 0;
+          cur.masked = 0;
+        }
+        const int buf = t % 3;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t / 3) & 1, wc))) {
           ok = false;
           break;
         }
@@ -500,10 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(trow + buf * 128 + 32 * h, pk);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // rescale this half of the running output once P.V of the previous
-          // tile landed.  S_t (ready here) was issued after P.V of tile t-2,
-          // so pv_done has completed t-1 or t phases and the parity test is
-          // exact.
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done, (t - 1) & 1, wc))) {
+          // tile landed.  pv_done[u & 1] completes once per P.V of tile u, so
+          // P.V t-1 is phase (t-1)>>1 of pv_done[(t-1) & 1]; the phase before
+          // it (P.V t-3) has completed because S_t, ready here, was issued
+          // after P.V t-3, so the parity test is exact.
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, wc))) {
             ok = false;
             break;
           }
@@ -511,11 +537,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(trow + 256 + DH * h + c0, o);
+            tmem_ld32(trow + kTmemO + DH * h + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(trow + 256 + DH * h + c0, o);
+            tmem_st32(trow + kTmemO + DH * h + c0, o);
           }
         }
         tmem_wait_st();
@@ -531,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t o[DH / 32][32];
 #pragma unroll
-      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld32(trow + 256 + DH * h + 32 * c0, o[c0]);
+      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld32(trow + kTmemO + DH * h + 32 * c0, o[c0]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&o_free);
