@@ -336,10 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0, t0 = 0;   // items so far, global index of the item's first tile
     const uint32_t tO = tmem + kTmemO;
     const uint32_t qaddr = sbase + C::Q_OFF;
-    // S_t = Q K_t^T into S buffer t % 3
-    auto issue_s = [&](int t, bool last) -> bool {
+    // S_t = Q K_t^T into S buffer t % 3 (k_ready: K_t is known to have landed)
+    auto issue_s = [&](int t, bool last, bool k_ready) -> bool {
       const int s = t % kNSK;
-      if (!warp_wait(&k_full[s], (t / kNSK) & 1, wc)) return false;
+      if (!k_ready && !warp_wait(&k_full[s], (t / kNSK) & 1, wc)) return false;
       tc_fence_after();
       const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
       const uint32_t tS = tmem + (t % 3) * 128;
@@ -359,13 +359,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nt = I.ntiles;
       if (!warp_wait(&q_full, n & 1, wc)) break;
       tc_fence_after();
-      for (int j = 0; ok && j < nt && j < 2; ++j) ok = issue_s(t0 + j, j == nt - 1);
+      for (int j = 0; ok && j < nt && j < 2; ++j) ok = issue_s(t0 + j, j == nt - 1, false);
       for (int j = 0; ok && j < nt; ++j) {
-        if (j + 2 < nt && !(ok = issue_s(t0 + j + 2, j + 2 == nt - 1))) break;
+        const int tp = t0 + j, sp = tp % kNSV, pb = tp % 3, ts = tp + 2;
+        const bool do_s = j + 2 < nt, first_pv = j == 0 && n > 0;
+        // Test everything this step needs at once, without blocking: the
+        // tests' latencies overlap, and the MMA queue is shallow, so a chain
+        // of waits here would leave the tensor pipe idle.  Blocking waits
+        // remain only for what is not ready yet.
+        uint32_t r = (do_s ? (uint32_t)mbar_test(&k_full[ts % kNSK], (ts / kNSK) & 1) : 1u) |
+                     ((uint32_t)mbar_test(&p_full[pb], (tp / 3) & 1) << 1) |
+                     ((uint32_t)mbar_test(&v_full[sp], (tp / kNSV) & 1) << 2) |
+                     ((first_pv ? (uint32_t)mbar_test(&o_free, (n - 1) & 1) : 1u) << 3);
+        r = __reduce_and_sync(0xFFFFFFFFu, r);
+        if (do_s && !(ok = issue_s(ts, ts == t0 + nt - 1, (r & 1u) != 0))) break;
         // O (+)= P_tp V_tp
-        const int tp = t0 + j, sp = tp % kNSV, pb = tp % 3;
-        if (!warp_wait(&p_full[pb], (tp / 3) & 1, wc) || !warp_wait(&v_full[sp], (tp / kNSV) & 1, wc) ||
-            (j == 0 && n > 0 && !warp_wait(&o_free, (n - 1) & 1, wc))) {
+        if ((!(r & 2u) && !warp_wait(&p_full[pb], (tp / 3) & 1, wc)) ||
+            (!(r & 4u) && !warp_wait(&v_full[sp], (tp / kNSV) & 1, wc)) ||
+            (!(r & 8u) && !warp_wait(&o_free, (n - 1) & 1, wc))) {
           ok = false;
           break;
         }

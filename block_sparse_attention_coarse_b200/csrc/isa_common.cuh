@@ -106,6 +106,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` of `bar` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared state of the bounded waits of one CTA.
 struct WaitCtl {
   volatile int* abort;       // shared-memory flag: some wait of this CTA ran out
@@ -316,11 +329,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // 2^x for a pair of floats on the FMA/ALU pipes (no MUFU): x = n + f with
 // n = round(x), f in [-1/2, 1/2]; 2^f by a cubic with 7.5e-5 maximum relative
 // error (relative-minimax fit by Lawson's algorithm, see fit_exp2_poly.py);
-// 2^n by adding n to the exponent field.  x is clamped at -126, so very
-// negative inputs (and -inf) give a denormal below 1.2e-38 instead of 0.
+// 2^n by adding n to the exponent field.  x is clamped to [-126, 126]: very
+// negative inputs (and -inf) give a denormal below 1.2e-38 instead of 0, and
+// large ones saturate near 2^126 instead of wrapping the exponent field.
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
+  x.x = fminf(fmaxf(x.x, -126.f), 126.f);
+  x.y = fminf(fmaxf(x.y, -126.f), 126.f);
   const float2 magic = make_float2(12582912.f, 12582912.f);   // 1.5 * 2^23
   const float2 t = fadd2(x, magic);                              // n in the low mantissa bits
   const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
