@@ -215,6 +215,52 @@ def test_forward_dit14b_full_size(isa):
     check_case(isa, w, heads=heads, blocks_per_head=6)
 
 
+def test_forward_long65k_b32_full_size(isa):
+    """b = 32: four query blocks per 128-row tile and four kept blocks per KV
+    tile; 32768 + 32768 tokens, H=40, D=128 (2048 blocks per head)."""
+    w = named_workloads()["long65k_b32"]
+    heads = sorted({bh for bh, _ in sample_blocks(w, 3, 1)})
+    check_case(isa, w, heads=heads, blocks_per_head=6)
+
+
+def test_forward_d64_131k_full_size(isa):
+    """D = 64 at the longest sweep length: 65536 + 65536 tokens, H=40."""
+    w = named_workloads()["sweep_L131072_D64"]
+    heads = sorted({bh for bh, _ in sample_blocks(w, 2, 1)})
+    check_case(isa, w, heads=heads, blocks_per_head=5)
+
+
+def test_forward_alpha_f_075_full_size(isa):
+    """Three quarters of the blocks flat (most rows on the pooled path)."""
+    w = named_workloads()["long65k_af075"]
+    heads = sorted({bh for bh, _ in sample_blocks(w, 2, 1)})
+    check_case(isa, w, heads=heads, blocks_per_head=6)
+
+
+def test_dense_dit14b_full_size_sampled_rows(isa):
+    """isa_dense at the benchmarked size against the oracle's dense attention
+    on a seeded sample of rows of a few heads."""
+    w = named_workloads()["dit14b"]
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    out = isa.dense(q, k, v, p, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    out = out.float().cpu().numpy().reshape(w.BH, w.L, w.D)
+    lse = lse.cpu().numpy().reshape(w.BH, w.L)
+    g = np.random.default_rng(77)
+    for h in sorted(g.choice(w.BH, size=3, replace=False).tolist()):
+        rows = np.sort(g.choice(w.L, size=256, replace=False))
+        ref, ref_lse = O.dense_attention(*(bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb)),
+                                         1 / np.sqrt(w.D), rows=rows)
+        d = np.abs(out[h][rows] - ref)
+        assert d.max() <= OUT_MAX_ABS and d.mean() <= OUT_MEAN_ABS, (h, d.max(), d.mean())
+        assert np.abs(lse[h][rows] - ref_lse).max() <= 2e-2
+
+
 # ---------------------------------------------------------------------------
 # bounded waits
 # ---------------------------------------------------------------------------
