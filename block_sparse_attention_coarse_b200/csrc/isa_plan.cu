@@ -113,20 +113,39 @@ __global__ void __launch_bounds__(256) ctx_select_kernel(Dims dm, PlanPtrs pp) {
   int* kept = pp.kept + (size_t)bh * dm.T_kv;
   for (int i = tid; i < dm.K_sel; i += 256) pp.ctx_sel[(size_t)bh * dm.K_sel + i] = sel[i];
   for (int i = tid; i < dm.T_kv; i += 256) kept[i] = i < dm.T_src ? i : dm.T_src + sel[i - dm.T_src];
-  // bf16 pooled K and V of the kept blocks, zero rows up to T_kv_pad
-  const float* Vc = pp.Vc + (size_t)bh * dm.T * D;
-  __nv_bfloat16* Kp = pp.Kp + (size_t)bh * dm.T_kv_pad * D;
-  __nv_bfloat16* Vp = pp.Vp + (size_t)bh * dm.T_kv_pad * D;
-  for (int e = tid; e < dm.T_kv_pad * D; e += 256) {
-    const int r = e / D, d = e % D;
-    float kv = 0.f, vv = 0.f;
-    if (r < dm.T_kv) {
-      const int j = r < dm.T_src ? r : dm.T_src + sel[r - dm.T_src];
-      kv = Kc[(size_t)j * D + d];
-      vv = Vc[(size_t)j * D + d];
+}
+
+// ---------------------------------------------------------------------------
+// K2a': bf16 pooled K and V of the kept blocks (the keys and values of the
+// pooled terms), zero rows up to T_kv_pad.  grid (ceil(T_kv_pad/8), BH), 256
+// threads; warp w converts kept row 8*blockIdx.x + w, each lane D/32
+// consecutive columns.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) pooled_kv_kernel(Dims dm, PlanPtrs pp) {
+  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= dm.T_kv_pad) return;
+  constexpr int PER = D / 32;
+  float kv[PER], vv[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) kv[u] = vv[u] = 0.f;
+  if (r < dm.T_kv) {
+    const int j = pp.kept[(size_t)bh * dm.T_kv + r];
+    const float* kr = pp.Kc + ((size_t)bh * dm.T + j) * D + PER * lane;
+    const float* vr = pp.Vc + ((size_t)bh * dm.T + j) * D + PER * lane;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      kv[u] = kr[u];
+      vv[u] = vr[u];
     }
-    Kp[e] = __float2bfloat16_rn(kv);
-    Vp[e] = __float2bfloat16_rn(vv);
+  }
+  __nv_bfloat16* Kp = pp.Kp + ((size_t)bh * dm.T_kv_pad + r) * D + PER * lane;
+  __nv_bfloat16* Vp = pp.Vp + ((size_t)bh * dm.T_kv_pad + r) * D + PER * lane;
+#pragma unroll
+  for (int u = 0; u < PER; u += 2) {
+    *reinterpret_cast<__nv_bfloat162*>(Kp + u) = __floats2bfloat162_rn(kv[u], kv[u + 1]);
+    *reinterpret_cast<__nv_bfloat162*>(Vp + u) = __floats2bfloat162_rn(vv[u], vv[u + 1]);
   }
 }
 
@@ -265,9 +284,12 @@ __global__ void __launch_bounds__(256) split_kernel(Dims dm, PlanPtrs pp) {
 
 // ---------------------------------------------------------------------------
 // K2d: exact-block lists of the flat blocks.  grid (ceil(n_flat/8), BH),
-// 256 threads; warp w owns flat block 8*blockIdx.x + w.  Scores of all kept
-// blocks for the 8 rows are built in shared memory (each warp computes whole
-// dot products for a strided set of kept blocks), then each warp selects.
+// 256 threads; warp w owns flat block 8*blockIdx.x + w.  The kept rows of Kc
+// stream through shared memory 32 at a time (row stride D+4 floats, so the
+// 16-byte reads of eight lanes on eight different rows hit different banks);
+// lane l of warp w forms the whole dot product of flat row w with kept row
+// l of the chunk.  The scores of all kept blocks for the 8 rows are kept in
+// shared memory, then each warp selects its row's exact blocks.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
@@ -283,21 +305,27 @@ __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
     qrows[e] = f < dm.n_flat ? Qc[(size_t)pp.flat[(size_t)bh * dm.n_flat + f] * D + d] : 0.f;
   }
   __syncthreads();
-  constexpr int PER = D / 32;
-  for (int kk = warp; kk < dm.T_kv; kk += 8) {
-    const float* kr = Kc + (size_t)kept[kk] * D;
-    float kv[PER];
-#pragma unroll
-    for (int u = 0; u < PER; ++u) kv[u] = kr[lane + 32 * u];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float s = 0.f;
-#pragma unroll
-      for (int u = 0; u < PER; ++u) s = fmaf(qrows[r * D + lane + 32 * u], kv[u], s);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0) sc[r * dm.T_kv + kk] = s * dm.scale;
+  constexpr int KS = D + 4;         // padded row stride of the Kc chunk
+  float* kch = sc + 8 * dm.T_kv;    // [32][KS]
+  const float4* q4 = reinterpret_cast<const float4*>(qrows + warp * D);
+  for (int k0 = 0; k0 < dm.T_kv; k0 += 32) {
+    __syncthreads();   // the previous chunk is consumed
+    for (int e = tid; e < 32 * (D / 4); e += 256) {
+      const int r = e / (D / 4), c4 = e % (D / 4);
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + r < dm.T_kv) w = reinterpret_cast<const float4*>(Kc + (size_t)kept[k0 + r] * D)[c4];
+      *reinterpret_cast<float4*>(kch + r * KS + 4 * c4) = w;
     }
+    __syncthreads();
+    const float4* k4 = reinterpret_cast<const float4*>(kch + lane * KS);
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; c4 += 2) {
+      const float4 a = q4[c4], b = k4[c4], a1 = q4[c4 + 1], b1 = k4[c4 + 1];
+      s0 = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, s0))));
+      s1 = fmaf(a1.x, b1.x, fmaf(a1.y, b1.y, fmaf(a1.z, b1.z, fmaf(a1.w, b1.w, s1))));
+    }
+    if (k0 + lane < dm.T_kv) sc[warp * dm.T_kv + k0 + lane] = (s0 + s1) * dm.scale;
   }
   __syncthreads();
   const int f = f0 + warp;
@@ -312,7 +340,9 @@ __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
 // host-side launchers (called from isa_api.cu)
 // ---------------------------------------------------------------------------
 static size_t rowstats_smem(int D) { return sizeof(float) * 2 * 64 * (D + 4); }
-static size_t exact_kernel_smem(const Dims& dm) { return sizeof(float) * 8 * ((size_t)dm.D + dm.T_kv); }
+static size_t exact_kernel_smem(const Dims& dm) {
+  return sizeof(float) * (8 * ((size_t)dm.D + dm.T_kv) + 32 * ((size_t)dm.D + 4));
+}
 
 template <int D>
 static cudaError_t launch_plan_d(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
@@ -325,6 +355,8 @@ static cudaError_t launch_plan_d(const Dims& dm, const void* q, const void* k, c
   if (e != cudaSuccess) return e;
   const size_t sm_ctx = sizeof(float) * (D + dm.T_ctx) + sizeof(int) * dm.K_sel;
   ctx_select_kernel<D><<<dm.BH, 256, sm_ctx, st>>>(dm, pp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  pooled_kv_kernel<D><<<dim3((dm.T_kv_pad + 7) / 8, dm.BH), 256, 0, st>>>(dm, pp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   rowstats_kernel<D><<<dim3((dm.T + 63) / 64, dm.BH), 256, rowstats_smem(D), st>>>(dm, pp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -346,9 +378,10 @@ cudaError_t prepare_plan_kernels() {
   if ((e = cudaFuncSetAttribute(rowstats_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)rowstats_smem(128))) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(exact_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(sizeof(float) * 8 * (64 + kMaxTkv)))) != cudaSuccess) return e;
+                                (int)(sizeof(float) * (8 * (64 + kMaxTkv) + 32 * (64 + 4))))) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(exact_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(sizeof(float) * 8 * (128 + kMaxTkv)))) != cudaSuccess) return e;
+                                (int)(sizeof(float) * (8 * (128 + kMaxTkv) + 32 * (128 + 4))))) != cudaSuccess)
+    return e;
   if ((e = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 3 * kMaxT * 4)) !=
       cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(ctx_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
