@@ -356,7 +356,7 @@ def run_gpu(args, w: Workload):
         "roofline": {"kernel": "attn_kernel (isa_forward)", "bound": "tensor", "achieved": achieved,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
                      "peak_kind": f"bf16 sustained ({peak_src})"},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 7 * args.steps,   # isa_plan: 6 kernels; isa_forward: 1
         "clocks": clk.summary(),
         "device_status": status,
     }
