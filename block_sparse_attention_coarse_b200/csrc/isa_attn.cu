@@ -22,8 +22,9 @@
 //   warp 0 lane 0 : TMA producer of the Q tile and the K tiles (kNSK stages)
 //   warp 1        : allocates TMEM; runs the MMA loop as one converged warp,
 //                   one elected lane issuing each tcgen05.mma / commit
-//   warps 2..9    : softmax / correction / epilogue; each query row is
-//                   handled by two threads (64 columns of the S tile each)
+//   warps 2..9    : softmax / correction / epilogue; each warp owns 16 query
+//                   rows, each row split between threads t and t+16 of the
+//                   warp (64 columns of the S tile each)
 //   warp 10 lane 0: TMA producer of the V tiles (kNSV stages)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+D).
 // S of tile t lives in buffer t % 3, so S runs two tiles ahead of P.V.  P (bf16)
@@ -206,6 +207,27 @@ __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, 
   return m;
 }
 
+// TMEM access of 16 lanes with the columns split between the two half warps
+// (the .16x32bx2 shape): thread t < 16 reaches lane base+t, columns
+// [c, c+32); thread t >= 16 reaches lane base+t-16, columns [c+SPLIT,
+// c+SPLIT+32).  So both 64-column halves of a row sit in one warp.
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
+      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+      : ISA_R32(r)
+      : "r"(taddr), "n"(SPLIT));
+}
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%"
+      "17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr),
+      "n"(SPLIT), ISA_W32(r)
+      : "memory");
+}
+
 // Warp-uniform bounded wait: every lane waits, the warp agrees on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, w));
@@ -221,9 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[kNSK], k_empty[kNSK], v_full[kNSV], v_empty[kNSV];
   __shared__ __align__(8) uint64_t s_full[3], p_full[3], pv_done[2], o_ready, o_free, drain_bar, inject_bar;
-  __shared__ __align__(8) uint64_t pair_max[4], pair_sum[4];   // the two softmax warps of one lane quarter
-  __shared__ float xmax[3][128][2];   // per S buffer, row, half: raw row maximum of the half
-  __shared__ float xsum[128][2];      // per row, half: softmax normaliser of the half
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -250,10 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&pv_done[1], 1);
     mbar_init(&o_ready, 1);
     mbar_init(&o_free, 256);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&pair_max[i], 64);
-      mbar_init(&pair_sum[i], 64);
-    }
     mbar_init(&drain_bar, 1);
     mbar_init(&inject_bar, 1);
     abort_flag = 0;
@@ -399,14 +414,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------ softmax
-    // Warps 2..9.  Two warps share each TMEM lane quarter (tcgen05.ld reaches
-    // lanes 32*(warp%4)..+31): half h = 0 takes columns 0..63 of the S tile,
-    // h = 1 columns 64..127, of the same 32 query rows.  The halves agree on
-    // the row maximum every tile through shared memory, keep separate
-    // partial normalisers, and combine them in the epilogue.
-    const int quarter = warp & 3, h = (warp - 2) >> 2;
-    const int row = quarter * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    // Warps 2..9.  Two warps share each TMEM lane quarter (tcgen05 access
+    // reaches lanes 32*(warp%4)..+31): warp half hw takes lanes 16*hw..+15 of
+    // the quarter, i.e. 16 query rows.  Thread t < 16 holds columns 0..63 of
+    // row t of the group (h = 0), thread t+16 columns 64..127 of the same row
+    // (h = 1): the row maximum is one shuffle, the two partial normalisers are
+    // added in the epilogue, and the two warps never wait for each other.
+    const int quarter = warp & 3, hw = (warp - 2) >> 2, h = lane >> 4;
+    const int row = quarter * 32 + hw * 16 + (lane & 15);
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32 + hw * 16) << 16);   // first lane of the group
     const int g_r = row / R, rr = row % R;
     const float sl2 = a.sl2;
     const float log2b = __log2f((float)a.b);
@@ -466,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t sr[2][32];
-        tmem_ld32(trow + buf * 128 + 64 * h, sr[0]);
-        tmem_ld32(trow + buf * 128 + 64 * h + 32, sr[1]);
+        tmem_ld16x2_32<64>(trow + buf * 128, sr[0]);        // columns 64h + 0..31
+        tmem_ld16x2_32<64>(trow + buf * 128 + 32, sr[1]);   // columns 64h + 32..63
         tmem_wait_ld();
         float s[64];
 #pragma unroll
@@ -489,14 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
         const float mh = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
-        xmax[buf][row][h] = mh;
-        mbar_arrive(&pair_max[quarter]);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pair_max[quarter], t & 1, wc))) {
-          ok = false;
-          break;
-        }
         const float bias = cur.pooled ? log2b : 0.f;
-        const float mx = fmaxf(mh, xmax[buf][row][h ^ 1]) * sl2 + bias;
+        const float mx = fmaxf(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 16)) * sl2 + bias;   // whole row
         const bool need = mx > m_run + kRescaleLog2;
         const float m_new = need ? mx : m_run;
         const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
@@ -533,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 a03 = fadd2(a01, a23);
         l_run = l_run * alpha + (a03.x + a03.y);
         m_run = m_new;
-        tmem_st32(trow + buf * 128 + 32 * h, pk);
+        tmem_st16x2_32<32>(trow + buf * 128, pk);   // P keys 64h..64h+63 -> columns 32h..32h+31
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // rescale this half of the running output once P.V of the previous
           // tile landed.  pv_done[u & 1] completes once per P.V of tile u, so
@@ -548,11 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(trow + kTmemO + DH * h + c0, o);
+            tmem_ld16x2_32<DH>(trow + kTmemO + c0, o);   // columns DH*h + c0..+31
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(trow + kTmemO + DH * h + c0, o);
+            tmem_st16x2_32<DH>(trow + kTmemO + c0, o);
           }
         }
         tmem_wait_st();
@@ -562,20 +572,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: wait until every P.V of the item landed (a per-item barrier:
       // pv_done may still be two phases behind here, because the last tile's
-      // S MMA was issued before the second-to-last P.V), combine the two
-      // halves' normalisers, normalise and write this half of each row
+      // S MMA was issued before the second-to-last P.V), add the partial
+      // normalisers of the row's two threads, normalise and write this
+      // thread's DH output columns of the row
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_ready, n & 1, wc))) break;
       tc_fence_after();
       uint32_t o[DH / 32][32];
 #pragma unroll
-      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld32(trow + kTmemO + DH * h + 32 * c0, o[c0]);
+      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld16x2_32<DH>(trow + kTmemO + 32 * c0, o[c0]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&o_free);
-      xsum[row][h] = l_run;
-      mbar_arrive(&pair_sum[quarter]);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pair_sum[quarter], n & 1, wc))) break;
-      const float l_tot = l_run + xsum[row][h ^ 1];
+      const float l_tot = l_run + __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
       if (row_valid) {
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
