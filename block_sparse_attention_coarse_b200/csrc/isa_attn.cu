@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float log2b = __log2f((float)a.b);
     constexpr int DH = D / 2;           // output columns of this half
     int n = 0, t = 0;
-    bool ok = true;
+    bool ok = true, s_ready = false;   // s_ready: S of tile t known complete
     for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
       const Item I = decode_item<G>(a, it);
       const int2 qs = q_span<R>(a, I, g_r);
@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           cur.masked = 0;
         }
         const int buf = t % 3;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t / 3) & 1, wc))) {
+        if (!s_ready && !__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t / 3) & 1, wc))) {
           ok = false;
           break;
         }
@@ -512,6 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
         const float alpha = need ? ex2(m_run - m_ref) : 1.f;
         const float neg = bias - m_ref;
+        // Is S of the next tile (t+1, possibly the next item's first) there
+        // already?  The test's latency overlaps the exponentials below, and a
+        // set phase stays set until the softmax has consumed that tile.
+        const bool s_next = mbar_test(&s_full[(t + 1) % 3], ((t + 1) / 3) & 1);
         // p = 2^(s * scale*log2e + bias - m_ref) in pairs; bf16 P for the MMA
         float2 acc[4];
 #pragma unroll
@@ -568,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[buf]);
+        s_ready = __all_sync(0xFFFFFFFFu, s_next);
       }
       if (!ok) break;
       // epilogue: wait until every P.V of the item landed (a per-item barrier:
