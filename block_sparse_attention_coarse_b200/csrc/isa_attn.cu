@@ -40,8 +40,10 @@ constexpr int kNSV = 2;             // V pipeline stages
 constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
 constexpr uint32_t kTmemO = 384;    // TMEM column of O (after three 128-column S buffers)
 // Exponentials of column pairs p with bit (p % 8) set go through the cubic on
-// the FMA pipe, the rest through MUFU (2 of 8).
-constexpr uint32_t kPolyPairs = 0x11u;
+// the FMA pipe, the rest through MUFU.  All on MUFU measured fastest at both
+// D=128 and D=64 (the FMA and ALU pipes are the more contended ones here;
+// 1, 2, 3 and 4 pairs of 8 on the cubic were 1-6 % slower).
+constexpr uint32_t kPolyPairs = 0x00u;
 
 template <int D, int R>
 struct Cfg {
