@@ -352,18 +352,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.inject) ok = warp_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
     int n = 0, t0 = 0;   // items so far, global index of the item's first tile
     const uint32_t tO = tmem + kTmemO;
-    const uint32_t qaddr = sbase + C::Q_OFF;
+    // Descriptors are built once per operand tile; the per-K-step offsets are
+    // added to the start-address field (address / 16, 14 bits: shared memory
+    // is below 256 KB, so the addition never carries out of the field).
+    const uint64_t qdesc = smem_desc_sw128(sbase + C::Q_OFF, 16, 1024);
     // S_t = Q K_t^T into S buffer t % 3 (k_ready: K_t is known to have landed)
     auto issue_s = [&](int t, bool last, bool k_ready) -> bool {
       const int s = t % kNSK;
       if (!k_ready && !warp_wait(&k_full[s], (t / kNSK) & 1, wc)) return false;
       tc_fence_after();
-      const uint32_t kaddr = sbase + C::K_OFF + s * C::TILE;
+      const uint64_t kdesc = smem_desc_sw128(sbase + C::K_OFF + s * C::TILE, 16, 1024);
       const uint32_t tS = tmem + (t % 3) * 128;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t o = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-        mma_ss_elect(tS, smem_desc_sw128(qaddr + o, 16, 1024), smem_desc_sw128(kaddr + o, 16, 1024), C::ID_S, ks > 0);
+        const uint32_t o = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tS, qdesc + o, kdesc + o, C::ID_S, ks > 0);
       }
       issued = true;
       tc_commit_elect(&s_full[t % 3]);
@@ -398,10 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t vaddr = sbase + C::V_OFF + sp * C::TILE;
+        const uint64_t vdesc = smem_desc_sw128(sbase + C::V_OFF + sp * C::TILE, C::CHUNK, 1024);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts_elect(tO, tmem + pb * 128 + ks * 8, smem_desc_sw128(vaddr + ks * 2048, C::CHUNK, 1024), C::ID_O,
+          mma_ts_elect(tO, tmem + pb * 128 + ks * 8, vdesc + (uint64_t)(ks * 2048 >> 4), C::ID_O,
                        (j > 0 || ks > 0) ? 1u : 0u);
         tc_commit_elect(&v_empty[sp]);
         tc_commit_elect(&pv_done[tp & 1]);
