@@ -351,3 +351,36 @@ def isa_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, p: Params):
     if single:
         out, lse = out[0], lse[0]
     return out, lse, plans
+
+
+# ----------------------------------------------------------------------------
+# decoupled rotary position embedding (applied to Q and K before step (1))
+# ----------------------------------------------------------------------------
+
+def rope_decoupled(x: np.ndarray, L_src: int, L_ctx: int, base: float = 10000.0) -> np.ndarray:
+    """Rotary position embedding with per-segment positions ([T] "Decoupled
+    RoPE": the reference video's positions restart at 0 instead of continuing
+    after the source video; [R] innovation (d): source and context each encode
+    positions from 0).
+
+    x: [..., L, D] with L = L_src + L_ctx.  Token l has position l in the
+    source segment and l - L_src in the context segment.  Reading of what the
+    pages leave open: one-dimensional RoPE over the token index, frequencies
+    theta_i = base^(-2i/D) for i = 0..D/2-1, pair i = components (2i, 2i+1)
+    rotated by the angle position * theta_i:
+        y[2i]   = x[2i] cos(a) - x[2i+1] sin(a)
+        y[2i+1] = x[2i] sin(a) + x[2i+1] cos(a).
+    fp64 throughout.
+    """
+    x = np.asarray(x, np.float64)
+    L, D = x.shape[-2], x.shape[-1]
+    assert L == L_src + L_ctx and D % 2 == 0
+    pos = np.concatenate([np.arange(L_src), np.arange(L_ctx)]).astype(np.float64)
+    theta = base ** (-2.0 * np.arange(D // 2) / D)
+    ang = pos[:, None] * theta[None, :]                     # [L, D/2]
+    c, s = np.cos(ang), np.sin(ang)
+    xe, xo = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = xe * c - xo * s
+    y[..., 1::2] = xe * s + xo * c
+    return y

@@ -393,3 +393,64 @@ def test_flat_path_is_convex_combination():
     p = O.Params(D=D, L_src=L_src, L_ctx=L_ctx, block=b, alpha_f=1.0, alpha_ns=0.1)
     out, _, _ = O.isa_forward(q, k, v, p)
     assert np.all(out <= v.max(axis=0) + 1e-12) and np.all(out >= v.min(axis=0) - 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# decoupled RoPE
+# ---------------------------------------------------------------------------
+
+def test_rope_position_zero_is_identity_in_both_segments():
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(9 + 6, 16))
+    y = O.rope_decoupled(x, 9, 6)
+    assert np.array_equal(y[0], x[0]) and np.array_equal(y[9], x[9])
+    assert not np.allclose(y[1], x[1])
+
+
+def test_rope_preserves_each_pair_norm():
+    rng = np.random.default_rng(6)
+    x = rng.normal(size=(3, 40, 32))
+    y = O.rope_decoupled(x, 25, 15)
+    nx = np.hypot(x[..., 0::2], x[..., 1::2])
+    ny = np.hypot(y[..., 0::2], y[..., 1::2])
+    assert np.abs(nx - ny).max() < 1e-12
+
+
+def test_rope_scores_depend_only_on_the_position_offset():
+    """Rotations compose: <R(m) q, R(n) k> is a function of n - m.  The same q
+    and k placed at (m, n) and at (m + s, n + s) give the same score."""
+    rng = np.random.default_rng(7)
+    D, L = 16, 50
+    q0, k0 = rng.normal(size=D), rng.normal(size=D)
+    for m, n, s in ((2, 9, 13), (0, 31, 7), (20, 3, 25)):
+        x = np.zeros((2, L, D))
+        x[0, m], x[1, n] = q0, k0
+        x[0, m + s], x[1, n + s] = q0, k0
+        y = O.rope_decoupled(x, L, 0)
+        a = y[0, m] @ y[1, n]
+        b = y[0, m + s] @ y[1, n + s]
+        assert abs(a - b) < 1e-10, (m, n, s, a, b)
+
+
+def test_rope_context_positions_restart_at_zero():
+    """A context token at segment position j is rotated exactly like a source
+    token at position j (not L_src + j)."""
+    rng = np.random.default_rng(8)
+    L_src, L_ctx, D = 30, 12, 8
+    x = rng.normal(size=(L_src + L_ctx, D))
+    x[L_src:] = x[:L_ctx]
+    y = O.rope_decoupled(x, L_src, L_ctx)
+    assert np.abs(y[L_src:] - y[:L_ctx]).max() < 1e-15
+
+
+def test_rope_rotation_angle_per_position_step():
+    """Measured with atan2: pair i = components (2i, 2i+1) turns
+    counter-clockwise by base^(-2i/D) radians per position step."""
+    D, L, base = 8, 6, 10000.0
+    x = np.zeros((L, D))
+    x[:, 0::2] = 1.0                  # every pair starts on the positive first axis
+    y = O.rope_decoupled(x, L, 0, base)
+    for i in range(D // 2):
+        ang = np.arctan2(y[:, 2 * i + 1], y[:, 2 * i])
+        step = np.angle(np.exp(1j * np.diff(ang)))
+        assert np.allclose(step, base ** (-2.0 * i / D), atol=1e-12), (i, step)
