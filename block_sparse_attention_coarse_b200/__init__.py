@@ -36,7 +36,7 @@ ISA_ERR_DEVICE_TIMEOUT = 5
 EXPORTS = (
     "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
-    "isa_forward_static",
+    "isa_forward_static", "isa_rope_workspace_size", "isa_rope",
 )
 
 
@@ -91,6 +91,8 @@ def load_library() -> ctypes.CDLL:
     lib.isa_set_fault_injection.argtypes = [ctypes.c_int32]
     lib.isa_forward_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.isa_forward_static.restype = ctypes.c_int
+    lib.isa_rope_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.isa_rope.argtypes = [P, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]
     for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
                  "isa_set_wait_timeout_ns", "isa_set_fault_injection"):
         getattr(lib, name).restype = ctypes.c_int
@@ -207,16 +209,41 @@ def plan_view(p: Params, ws: torch.Tensor) -> Dict[str, object]:
     return out
 
 
+def rope_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().isa_rope_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def rope(q: torch.Tensor, k: torch.Tensor, p: Params, base: float = 10000.0, inplace: bool = False,
+         ws: Optional[torch.Tensor] = None, stream=None):
+    """Decoupled rotary position embedding of q and k (positions restart at 0
+    in the context segment); returns the rotated (q, k), new tensors unless
+    `inplace`."""
+    _check_qkv(q, k, k, p)
+    qo, ko = (q, k) if inplace else (torch.empty_like(q), torch.empty_like(k))
+    if ws is None:
+        ws = torch.empty(rope_workspace_size(p), dtype=torch.uint8, device=q.device)
+    _check(load_library().isa_rope(ctypes.byref(p), float(base), q.data_ptr(), k.data_ptr(), qo.data_ptr(),
+                                   ko.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return qo, ko
+
+
 def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,
-                  device=None) -> torch.Tensor:
-    """The user-level call: plan + forward.  CUDA inputs stay on the device;
-    CPU inputs (pinned for overlap) are copied in and the output is copied
-    back to a pinned CPU tensor on the current stream."""
+                  device=None, rope_base: Optional[float] = None) -> torch.Tensor:
+    """The user-level call: plan + forward, after the decoupled RoPE of q and
+    k when `rope_base` is given.  CUDA inputs stay on the device; CPU inputs
+    (pinned for overlap) are copied in and the output is copied back to a
+    pinned CPU tensor on the current stream."""
     if q.is_cuda:
+        if rope_base is not None:
+            q, k = rope(q, k, p, rope_base)
         ws = plan(q, k, v, p, ws)
         return forward(q, k, v, ws, p)
     dev = torch.device(device or "cuda")
     qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    if rope_base is not None:
+        qd, kd = rope(qd, kd, p, rope_base, inplace=True)
     ws = plan(qd, kd, vd, p, ws)
     od = forward(qd, kd, vd, ws, p)
     out = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)

@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu"]
+SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu", "isa_rope.cu"]
 LIB = os.path.join(HERE, "libisa.so")
 HEADERS = [os.path.join(CSRC, "isa_common.cuh"), os.path.join(ROOT, "include", "isa.h")]
 

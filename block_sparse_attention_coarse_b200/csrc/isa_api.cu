@@ -348,6 +348,32 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
   return run_attention(d, 1, q, k, v, nullptr, out, lse, status, st);
 }
 
+isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if (!bytes) return fail(ISA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = rope_table_bytes(d);
+  return ISA_OK;
+}
+
+isa_status isa_rope(const isa_params* p, float base, const void* q, const void* k, void* q_out, void* k_out,
+                    void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if (!(base > 1.f) || !std::isfinite(base)) return fail(ISA_ERR_INVALID_ARG, "base must be finite and > 1");
+  if ((s = check_ptr(q, "q", 16)) != ISA_OK || (s = check_ptr(k, "k", 16)) != ISA_OK ||
+      (s = check_ptr(q_out, "q_out", 16)) != ISA_OK || (s = check_ptr(k_out, "k_out", 16)) != ISA_OK ||
+      (s = check_ptr(ws, "workspace", 16)) != ISA_OK)
+    return s;
+  const size_t need = rope_table_bytes(d);
+  if (ws_bytes < need) return fail(ISA_ERR_WORKSPACE, "rope workspace has %zu bytes, needs %zu", ws_bytes, need);
+  cudaError_t e = launch_rope(d, (double)base, q, k, q_out, k_out, ws, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  return ISA_OK;
+}
+
 const char* isa_last_error(void) { return g_last_error.c_str(); }
 
 const char* isa_version(void) { return "isa-b200 0.1 sm_100a"; }

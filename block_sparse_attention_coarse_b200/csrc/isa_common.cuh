@@ -59,6 +59,9 @@ cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void
                         cudaStream_t st);
 cudaError_t prepare_plan_kernels();
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
+size_t rope_table_bytes(const Dims& d);
+cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
+                        int sm_count, cudaStream_t st);
 void set_last_error(const char* msg);
 
 constexpr int kMaxT = 8192;      // blocks per head

@@ -159,6 +159,30 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
 isa_status isa_forward_static(const isa_params* p, const void* q, const void* k, const void* v, void* out,
                               float* lse, void* stream);
 
+/* Workspace of isa_rope: the cos/sin table, max(L_src, L_ctx) * D/2 float
+ * pairs (8 bytes each). */
+isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes);
+
+/* Decoupled rotary position embedding of Q and K, applied before isa_plan
+ * (techwalker.com article, "Decoupled RoPE": the reference video's position
+ * indices restart at 0 rather than continuing after the source video;
+ * summary card, innovation (d): source and context each encode positions
+ * from 0).  Token l has position l in the source segment [0, L_src) and
+ * l - L_src in the context segment.  The pages name no frequencies or
+ * pairing; this is one-dimensional RoPE over the token index with
+ * theta_i = base^(-2i/D), pair i = components (2i, 2i+1) rotated
+ * counter-clockwise by position * theta_i.
+ *   q, k         : device bf16 [B,H,L,D]
+ *   q_out, k_out : device bf16 [B,H,L,D]; may equal q, k (in place)
+ *   base         : > 1 (10000 is the usual value)
+ *   ws           : device, >= isa_rope_workspace_size bytes, 16-byte aligned;
+ *                  caller-owned, rewritten by every call
+ * Angles and the table are computed in double precision, the rotation in
+ * fp32 from bf16 inputs, rounded once to bf16 (round to nearest even).
+ * Stream-ordered; argument errors return before any launch. */
+isa_status isa_rope(const isa_params* p, float base, const void* q, const void* k, void* q_out, void* k_out,
+                    void* ws, size_t ws_bytes, void* stream);
+
 /* Thread-local description of the last error (never NULL). */
 const char* isa_last_error(void);
 

@@ -67,25 +67,34 @@ class HeadCheck:
         self.split_moved: List[int] = []      # blocks whose sharp/flat side differs
         self.exact_moved: List[int] = []      # flat blocks whose exact list differs
         self.errors: List[str] = []
+        self.outside_margin: List[str] = []   # set differences beyond the margins (inputs_equal=False)
 
 
-def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int) -> HeadCheck:
+def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int, inputs_equal: bool = True) -> HeadCheck:
     """Compares plan arrays of head `h` (host numpy copies of the plan view)
-    with the oracle plan `pl` under the margin rules."""
+    with the oracle plan `pl` under the margin rules.
+
+    inputs_equal=False: the two sides planned from inputs that may differ by
+    one bf16 rounding per element (each side applied its own position
+    embedding): value tolerances widen to cover that, and index-set
+    differences beyond the margins are recorded in `outside_margin` (to be
+    counted as moved blocks) instead of failing."""
     r = HeadCheck()
     T_src = pl.T_src
+    tol_pool, tol_imp, tol_energy = (1e-5, 1e-3, 1e-4) if inputs_equal else (2.0 ** -8, 2e-2, 2e-2)
+    margin_fail = r.errors if inputs_equal else r.outside_margin
     # pooled means (fp32 sums of bf16 values)
     for name, ref in (("Qc", pl.Qc), ("Kc", pl.Kc), ("Vc", pl.Vc)):
         got = gpu[name][h]
         err = np.abs(got - ref).max()
-        if err > 1e-5 * max(1.0, np.abs(ref).max()):
+        if err > tol_pool * max(1.0, np.abs(ref).max()):
             r.errors.append(f"{name} max err {err:.3g}")
     # context importance and selection
-    if np.abs(gpu["imp"][h] - pl.imp).max() > 1e-3 * max(1.0, np.abs(pl.imp).max()):
+    if np.abs(gpu["imp"][h] - pl.imp).max() > tol_imp * max(1.0, np.abs(pl.imp).max()):
         r.errors.append(f"imp max err {np.abs(gpu['imp'][h] - pl.imp).max():.3g}")
     ok, diff = topk_agrees(pl.imp / T_src, len(pl.ctx_sel), gpu["ctx_sel"][h], MARGIN_CTX)
     if not ok:
-        r.errors.append(f"ctx_sel outside margin: gpu {gpu['ctx_sel'][h].tolist()} oracle {pl.ctx_sel.tolist()}")
+        margin_fail.append(f"ctx_sel outside margin: gpu {gpu['ctx_sel'][h].tolist()} oracle {pl.ctx_sel.tolist()}")
     if list(gpu["ctx_sel"][h]) != sorted(gpu["ctx_sel"][h]):
         r.errors.append("ctx_sel not ascending")
     r.ctx_equal = np.array_equal(np.sort(gpu["ctx_sel"][h]), pl.ctx_sel)
@@ -94,7 +103,7 @@ def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int) -> HeadCheck:
         r.errors.append("kept list inconsistent with ctx_sel")
     # energy and split
     E = energy_from_oracle(pl)
-    if np.abs(gpu["energy"][h] - E).max() > 1e-4 * E.max():
+    if np.abs(gpu["energy"][h] - E).max() > tol_energy * E.max():
         r.errors.append(f"energy rel err {np.abs(gpu['energy'][h] - E).max() / E.max():.3g}")
     n_sharp = len(pl.sharp)
     sharp_gpu = gpu["sharp_ids"][h]
@@ -108,7 +117,7 @@ def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int) -> HeadCheck:
         boundary = 0.5 * (E[order[n_sharp - 1]] + E[order[n_sharp]])
         ok, _ = topk_agrees(E, n_sharp, sharp_gpu, MARGIN_SPLIT_REL * boundary)
         if not ok:
-            r.errors.append("sharp set outside margin")
+            margin_fail.append("sharp set outside margin")
     r.split_moved = sorted(set(sharp_gpu.tolist()).symmetric_difference(pl.sharp.tolist()))
     # exact lists, where the kept sets agree
     if r.ctx_equal:
@@ -119,7 +128,7 @@ def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int) -> HeadCheck:
             got = gpu["exact"][h][flat_pos_gpu[int(b)]]
             ok, diff = topk_agrees(pl.S[b, pl.kept], pl.exact.shape[1], got, MARGIN_EXACT)
             if not ok:
-                r.errors.append(f"exact list of block {b} outside margin")
+                margin_fail.append(f"exact list of block {b} outside margin")
             if list(got) != sorted(got):
                 r.errors.append("exact list not ascending")
             bits = gpu["exact_bits"][h][flat_pos_gpu[int(b)]].astype(np.uint32)

@@ -112,6 +112,23 @@ def test_null_and_misaligned_pointers_rejected_before_launch(isa):
     assert st == 1
 
 
+def test_rope_arguments_rejected_before_launch(isa):
+    """isa_rope checks the base, the pointers and the table size on the host
+    (fake device addresses: nothing may be launched)."""
+    lib = isa.load_library()
+    p = isa.make_params(1, 2, 64, 300, 100)
+    n = isa.rope_workspace_size(p)
+    assert n == 300 * 32 * 8          # max(L_src, L_ctx) * D/2 (cos, sin) float pairs
+    a = 1 << 20
+    assert lib.isa_rope(ctypes.byref(p), 1.0, a, a, a, a, a, n, None) == 1
+    assert b"base" in lib.isa_last_error()
+    assert lib.isa_rope(ctypes.byref(p), float("inf"), a, a, a, a, a, n, None) == 1
+    assert lib.isa_rope(ctypes.byref(p), 10000.0, a, a, a, None, a, n, None) == 1
+    assert b"k_out is NULL" in lib.isa_last_error()
+    assert lib.isa_rope(ctypes.byref(p), 10000.0, a, a + 8, a, a, a, n, None) == 1
+    assert lib.isa_rope(ctypes.byref(p), 10000.0, a, a, a, a, a, n - 1, None) == 3
+
+
 def test_binding_rejects_host_tensors(isa):
     import torch
     p = isa.make_params(1, 1, 64, 64, 64)
