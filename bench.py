@@ -12,8 +12,10 @@ bf16 inputs (the pages' video latents are not available).
 Prints one JSON line.  `value` is executed TFLOP/s over all ranks (4*D per
 query-token x key-column pair, pooled blocks one column each, plus 2*T*T*D
 per head for the coarse scores), `latency_ms` the per-step latency.  With
-N > 1 (torchrun) every rank runs its own copy of the workload (heads are
-independent; no data-path collective), timing is the max over ranks.
+N > 1 (torchrun) heads are independent, so there is no data-path
+collective: by default every rank runs its own copy of the workload (weak
+scaling); `--shard heads` splits the B*H heads of one workload across the
+ranks (strong scaling).  Timing is the max over ranks.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload (rank 0 only).
@@ -235,15 +237,26 @@ def run_gpu(args, w: Workload):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
 
-    # inputs: one full copy of the workload per rank, resident in HBM
-    wr = w.replace(seed=w.seed + 100 * rank) if world > 1 else w
-    qb, kb, vb = generate_bits(wr)
+    # inputs resident in HBM: replicas -> one full copy of the workload per
+    # rank (its own seed); heads -> this rank's contiguous slice of the B*H
+    # heads of one workload, drawn head by head with the workload's seed
+    if args.shard == "heads":
+        from block_sparse_attention_coarse_b200.shard import head_range
+        lo, hi = head_range(w.BH, rank, world)
+        if hi == lo:
+            raise SystemExit(f"--shard heads: {world} ranks for {w.BH} heads leaves rank {rank} without work")
+        qb, kb, vb = (x.reshape(1, hi - lo, w.L, w.D) for x in generate_bits(w, heads=range(lo, hi)))
+        B_r, H_r = 1, hi - lo
+    else:
+        wr = w.replace(seed=w.seed + 100 * rank) if world > 1 else w
+        qb, kb, vb = generate_bits(wr)
+        B_r, H_r = w.B, w.H
 
     def to_dev(x):
         return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
 
     q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
-    p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+    p = isa.make_params(B_r, H_r, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
     ws = isa.alloc_workspace(p, dev)
     out = torch.empty_like(q)
 
@@ -257,7 +270,7 @@ def run_gpu(args, w: Workload):
     view = isa.plan_view(p, ws)
     status = int(view["status"].item())
     flops = isa.executed_flops(p, view)
-    plan_flops = 2.0 * view["T"] ** 2 * w.D * w.BH
+    plan_flops = 2.0 * view["T"] ** 2 * w.D * B_r * H_r
     attn_flops = flops - plan_flops
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -286,7 +299,12 @@ def run_gpu(args, w: Workload):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
     ms_per_step = elapsed_ms / args.steps
-    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+    job_flops = flops                        # work of all ranks per step
+    if world > 1:
+        t = torch.tensor([flops], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        job_flops = float(t.item())
+    value = job_flops * args.steps / (elapsed_ms / 1e3) / 1e12
 
     # the dense kernel on the same inputs
     dense_ms = None
@@ -321,7 +339,7 @@ def run_gpu(args, w: Workload):
             t = torch.tensor([e2e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
-        e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(3 * q.numel() * 2), "d2h_bytes_per_step": int(res.numel() * 2),
                "ms_per_step": e2e_ms}
         del qh, kh, vh, res
@@ -340,14 +358,15 @@ def run_gpu(args, w: Workload):
     peak_burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
     hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
     T = int(view["T"])
-    plan_bytes = 3 * q.numel() * 2 + 3 * w.BH * T * w.D * 4
+    plan_bytes = 3 * q.numel() * 2 + 3 * B_r * H_r * T * w.D * 4
+    parallelism = "single" if world == 1 else (f"heads{world}" if args.shard == "heads" else f"replicas{world}")
     traffic = attn_traffic(w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "latency_ms": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded clustered generator, no trained weights)",
-        "config": {**describe(w), "parallelism": f"replicas{world}" if world > 1 else "single",
+        "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded clustered generator, no trained weights)",
+        "config": {**describe(w), "parallelism": parallelism, "heads_per_rank": B_r * H_r,
                    "l2": f"inputs {3 * q.numel() * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush)"},
         "plan_ms": plan_avg, "forward_ms": fwd_avg, "executed_tflop_per_step": flops / 1e12,
         "tflops_frac_sustained": achieved / peak_sus, "tflops_frac_burst": achieved / peak_burst,
@@ -380,6 +399,9 @@ def main():
     ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N>1: replicas = every rank runs the whole workload (weak scaling); "
+                         "heads = the ranks split the B*H heads of one workload (strong scaling)")
     args = ap.parse_args()
     w = named_workloads()[args.workload]
     if args.impl == "reference":
