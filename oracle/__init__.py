@@ -8,4 +8,5 @@ from .isa_oracle import (Params, HeadPlan, segment_blocks, pool, coarse_scores,
                          context_importance, topk_lower_index, softmax_rows, sharpness,
                          split_sharp_flat, plan_head, forward_head, dense_attention,
                          isa_forward, n_select, n_flat_blocks, n_exact_blocks,
-                         sharp_block, flat_block, rope_decoupled)
+                         sharp_block, flat_block, rope_decoupled,
+                         backward_head, isa_backward)

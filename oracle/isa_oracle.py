@@ -26,6 +26,8 @@ The oracle follows the steps in the order of [R] "Method steps in detail":
       block contributes exp(q Kc_j^T / sqrt(D)) * Vc_j weighted by its token
       count; one softmax normaliser over both parts
   (6) outputs return to token order (no gamma * O_coarse residual).
+The backward (``backward_head``, ``isa_backward``) differentiates steps
+(4)-(6) with the plan held fixed; see the note above ``backward_head``.
 
 Readings of points the pages leave open (every one is switchable where a
 second reading is plausible; the defaults are the ones the CUDA path uses):
@@ -384,3 +386,105 @@ def rope_decoupled(x: np.ndarray, L_src: int, L_ctx: int, base: float = 10000.0)
     y[..., 0::2] = xe * c - xo * s
     y[..., 1::2] = xe * s + xo * c
     return y
+
+
+# ----------------------------------------------------------------------------
+# backward of steps (4)-(6)
+# ----------------------------------------------------------------------------
+# [R] "Core method" and innovation (c), [T] "Decoupled RoPE" paragraph: the
+# method has a forward and a backward implementation and is trained end to
+# end.  The pages give no backward formulas; the reading here is the plain
+# one: the gradient of the step (4)-(6) output with respect to Q, K and V
+# with the plan held fixed.  The plan's choices (kept context blocks, the
+# sharp/flat split, the exact lists) are piecewise constant in the inputs and
+# carry no gradient; the pooled key/value means of the flat path are
+# functions of K and V (Kc_j = mean of the keys of block j), so their
+# gradient reaches every token of block j divided by n_j.  The count weight
+# n_j is a constant.
+
+def _weighted_average_grad(logits: np.ndarray, values: np.ndarray, log_weights: np.ndarray,
+                           dout: np.ndarray):
+    """Gradients of rows o = softmax(logits + log_weights) @ values.
+
+    Returns (dlogits, dvalues): with P the softmax and dP = dout values^T,
+    dlogits = P * (dP - rowsum(dout * o)) and dvalues = P^T dout.
+    """
+    z = logits + log_weights[None, :]
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    P = e / e.sum(axis=1, keepdims=True)
+    o = P @ values
+    dP = dout @ values.T
+    delta = (dout * o).sum(axis=1, keepdims=True)
+    return P * (dP - delta), P.T @ dout
+
+
+def backward_head(q, k, v, plan: HeadPlan, p: Params, dout, blocks: Optional[Sequence[int]] = None):
+    """(dq, dk, dv) [L, D] of one head for the loss sum(dout * out).
+
+    Same columns per query block as ``forward_head``: a sharp block sees
+    every token of the kept blocks; a flat block sees the tokens of its exact
+    blocks and one pooled column (Kc_j, Vc_j, log-weight ln n_j) per other
+    kept block.  The gradients of the pooled columns are gathered per block
+    and spread over the block's tokens with weight 1/n_j at the end.
+    ``blocks`` restricts the sum to those query blocks (their dq rows are
+    then complete; dk, dv hold only their share).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    dout = np.asarray(dout, np.float64)
+    s = p.s
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dKc, dVc = np.zeros((plan.T, p.D)), np.zeros((plan.T, p.D))
+    todo = range(plan.T) if blocks is None else blocks
+    flat_pos = {int(b): r for r, b in enumerate(plan.flat)}
+    for i in todo:
+        i = int(i)
+        rows = np.arange(plan.starts[i], plan.starts[i] + plan.counts[i])
+        if i not in flat_pos:
+            cols = _kept_tokens(plan, plan.kept)
+            dz, dvals = _weighted_average_grad((q[rows] @ k[cols].T) * s, v[cols], np.zeros(len(cols)), dout[rows])
+            dq[rows] += s * (dz @ k[cols])
+            dk[cols] += s * (dz.T @ q[rows])
+            dv[cols] += dvals
+            continue
+        ex_blocks = plan.kept[plan.exact[flat_pos[i]]]
+        pooled = np.array([j for j in plan.kept if j not in set(ex_blocks.tolist())], np.int64)
+        tok = _kept_tokens(plan, ex_blocks)
+        nt = len(tok)
+        logits = np.concatenate([q[rows] @ k[tok].T, q[rows] @ plan.Kc[pooled].T], axis=1) * s
+        values = np.concatenate([v[tok], plan.Vc[pooled]], axis=0)
+        logw = np.concatenate([np.zeros(nt), np.log(plan.counts[pooled].astype(np.float64))])
+        dz, dvals = _weighted_average_grad(logits, values, logw, dout[rows])
+        dq[rows] += s * (dz[:, :nt] @ k[tok] + dz[:, nt:] @ plan.Kc[pooled])
+        dk[tok] += s * (dz[:, :nt].T @ q[rows])
+        dv[tok] += dvals[:nt]
+        dKc[pooled] += s * (dz[:, nt:].T @ q[rows])
+        dVc[pooled] += dvals[nt:]
+    # Kc_j = (1/n_j) * sum of the keys of block j (and Vc_j likewise)
+    for j in range(plan.T):
+        t = slice(plan.starts[j], plan.starts[j] + plan.counts[j])
+        dk[t] += dKc[j] / plan.counts[j]
+        dv[t] += dVc[j] / plan.counts[j]
+    return dq, dk, dv
+
+
+def isa_backward(q, k, v, dout, p: Params):
+    """Backward over [B, H, L, D] (or [L, D]) fp64 inputs: plans each head
+    from (q, k, v) as ``isa_forward`` does and returns (dq, dk, dv)."""
+    q = np.asarray(q, np.float64)
+    single = q.ndim == 2
+    if single:
+        q, k, v, dout = q[None], np.asarray(k)[None], np.asarray(v)[None], np.asarray(dout)[None]
+    lead = q.shape[:-2]
+    flat = [np.asarray(x, np.float64).reshape(-1, p.L, p.D) for x in (q, k, v, dout)]
+    grads = [[], [], []]
+    for h in range(flat[0].shape[0]):
+        qh, kh, vh, dh = (x[h] for x in flat)
+        g = backward_head(qh, kh, vh, plan_head(qh, kh, vh, p), p, dh)
+        for a, b in zip(grads, g):
+            a.append(b)
+    out = [np.stack(g).reshape(*lead, p.L, p.D) for g in grads]
+    if single:
+        out = [x[0] for x in out]
+    return tuple(out)
