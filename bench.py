@@ -57,7 +57,7 @@ def attn_traffic(workload: str):
     None when the kernel source changed since the counters were taken."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "attn_traffic.txt")
-    src = os.path.join(ROOT, "block_sparse_attention_coarse_b200", "csrc", "isa_attn.cu")
+    csrc = os.path.join(ROOT, "block_sparse_attention_coarse_b200", "csrc")
     try:
         vals = {}
         for line in open(path):
@@ -65,7 +65,10 @@ def attn_traffic(workload: str):
             if "=" in line:
                 k, v = (x.strip() for x in line.split("=", 1))
                 vals[k] = v
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        h = hashlib.sha256()
+        for f in ("isa_attn.cu", "isa_items.cuh"):   # the kernel and its work-item helpers
+            h.update(open(os.path.join(csrc, f), "rb").read())
+        sha = h.hexdigest()
     except OSError:
         return None
     if vals.get("kernel_source_sha256") != sha or workload not in vals:
@@ -320,6 +323,35 @@ def run_gpu(args, w: Workload):
         torch.cuda.synchronize(dev)
         dense_ms = e0.elapsed_time(e1) / nd
 
+    # the backward (isa_backward) on the same plan: dq, dk, dv of sum(dout * out)
+    bwd = None
+    if not args.skip_backward:
+        from workloads import generate_dout_bits
+        if args.shard == "heads":
+            db = generate_dout_bits(w, heads=range(lo, hi)).reshape(1, hi - lo, w.L, w.D)
+        else:
+            db = generate_dout_bits(wr)
+        dout = to_dev(db)
+        lse = torch.empty(B_r, H_r, w.L, dtype=torch.float32, device=dev)
+        isa.forward(q, k, v, ws, p, out=out, lse=lse)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(isa.backward_workspace_size(p), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            isa.backward(q, k, v, ws, p, out, lse, dout, dq, dk, dv, bws)
+        torch.cuda.synchronize(dev)
+        nbk = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(nbk):
+            isa.backward(q, k, v, ws, p, out, lse, dout, dq, dk, dv, bws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        bwd_ms = e0.elapsed_time(e1) / nbk
+        # algorithmic work: five products per (query, column) pair against the forward's two
+        bwd = {"ms": bwd_ms, "tflops": 2.5 * attn_flops / (bwd_ms / 1e3) / 1e12, "launches_per_call": 5,
+               "flops_convention": "2.5 x the forward's attention FLOPs (5 vs 2 matrix products)"}
+        del dout, dq, dk, dv, bws, lse
+
     # end to end through the public API from pinned host memory
     e2e = None
     if not args.skip_e2e:
@@ -381,6 +413,8 @@ def run_gpu(args, w: Workload):
     }
     if e2e:
         line["e2e"] = e2e
+    if bwd:
+        line["backward"] = bwd
     if world == 1 and not args.skip_cpu:
         fl, secs, desc = oracle_sample(w)
         line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
@@ -399,6 +433,7 @@ def main():
     ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N>1: replicas = every rank runs the whole workload (weak scaling); "
                          "heads = the ranks split the B*H heads of one workload (strong scaling)")

@@ -12,7 +12,9 @@ Video Editing via In-Context Sparse Attention" (paper.rainbus.top summary,
 "Method steps in detail"):
   plan(...)    steps (1)-(3) + the exact-block choice of step (5)
   forward(...) steps (4)-(6), sharp and flat query blocks in one launch
+  backward(...) gradients of steps (4)-(6) with the plan held fixed
   dense(...)   the full attention that ISA replaces
+  IsaAttention torch.autograd.Function over plan + forward / backward
 """
 from __future__ import annotations
 
@@ -36,7 +38,7 @@ ISA_ERR_DEVICE_TIMEOUT = 5
 EXPORTS = (
     "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
-    "isa_forward_static", "isa_rope_workspace_size", "isa_rope",
+    "isa_forward_static", "isa_rope_workspace_size", "isa_rope", "isa_backward_workspace_size", "isa_backward",
 )
 
 
@@ -93,8 +95,11 @@ def load_library() -> ctypes.CDLL:
     lib.isa_forward_static.restype = ctypes.c_int
     lib.isa_rope_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.isa_rope.argtypes = [P, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]
+    lib.isa_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.isa_backward.argtypes = [P, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
-                 "isa_set_wait_timeout_ns", "isa_set_fault_injection"):
+                 "isa_set_wait_timeout_ns", "isa_set_fault_injection", "isa_rope_workspace_size", "isa_rope",
+                 "isa_backward_workspace_size", "isa_backward"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -227,6 +232,56 @@ def rope(q: torch.Tensor, k: torch.Tensor, p: Params, base: float = 10000.0, inp
     _check(load_library().isa_rope(ctypes.byref(p), float(base), q.data_ptr(), k.data_ptr(), qo.data_ptr(),
                                    ko.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
     return qo, ko
+
+
+def backward_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().isa_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ws: torch.Tensor, p: Params, out: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, dq: Optional[torch.Tensor] = None,
+             dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+             bws: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dq, dk, dv) of sum(dout * out) for the forward that produced
+    `out` and `lse` from (q, k, v) with the plan in `ws`."""
+    _check_qkv(q, k, v, p)
+    _check_qkv(out, dout, out, p)
+    L = p.L_src + p.L_ctx
+    if not lse.is_cuda or lse.dtype != torch.float32 or tuple(lse.shape) != (p.B, p.H, L) or not lse.is_contiguous():
+        raise IsaError(ISA_ERR_INVALID_ARG, f"lse must be contiguous float32 {(p.B, p.H, L)}")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv(dq, dk, dv, p)
+    if bws is None:
+        bws = torch.empty(backward_workspace_size(p), dtype=torch.uint8, device=q.device)
+    _check(load_library().isa_backward(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), ws.data_ptr(),
+                                       ws.numel(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                                       dk.data_ptr(), dv.data_ptr(), bws.data_ptr(), bws.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+class IsaAttention(torch.autograd.Function):
+    """ISA as a differentiable op: forward = plan + sparse attention (keeping
+    the plan, output and lse), backward = the library's backward with that
+    plan.  Inputs are contiguous bf16 CUDA tensors [B, H, L, D]."""
+
+    @staticmethod
+    def forward(ctx, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params) -> torch.Tensor:
+        ws = plan(q, k, v, p)
+        lse = torch.empty(p.B, p.H, p.L_src + p.L_ctx, dtype=torch.float32, device=q.device)
+        out = forward(q, k, v, ws, p, lse=lse)
+        ctx.save_for_backward(q, k, v, ws, out, lse)
+        ctx.p = p
+        return out
+
+    @staticmethod
+    def backward(ctx, dout: torch.Tensor):
+        q, k, v, ws, out, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, ws, ctx.p, out, lse, dout.contiguous())
+        return dq, dk, dv, None
 
 
 def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,

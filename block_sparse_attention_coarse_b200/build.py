@@ -16,9 +16,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu", "isa_rope.cu"]
+SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu", "isa_rope.cu", "isa_bwd.cu"]
 LIB = os.path.join(HERE, "libisa.so")
-HEADERS = [os.path.join(CSRC, "isa_common.cuh"), os.path.join(ROOT, "include", "isa.h")]
+HEADERS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
+    os.path.join(ROOT, "include", "isa.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

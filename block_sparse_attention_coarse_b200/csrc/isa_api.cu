@@ -159,6 +159,29 @@ isa_status ensure_init() {
   return ISA_OK;
 }
 
+}  // namespace
+
+namespace isa {
+// Makes the device that owns `ptr` current on the calling thread (binding its
+// primary context), so that a call from a thread that never selected a
+// device -- a framework's autograd worker, a thread pool -- encodes its
+// tensor maps and launches on the GPU that holds the data.
+isa_status bind_device_of(const void* ptr, const char* name) {
+  cudaPointerAttributes at{};
+  cudaError_t e = cudaPointerGetAttributes(&at, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, name);
+  }
+  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+    return fail(ISA_ERR_INVALID_ARG, "%s is not CUDA device memory", name);
+  if ((e = cudaSetDevice(at.device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  return ISA_OK;
+}
+}  // namespace isa
+
+namespace {
+
 // rows x D bf16, box of 64 columns x box_rows rows, 128-byte swizzle
 isa_status make_map(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows, const char* name) {
   cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
@@ -243,7 +266,7 @@ isa_status isa_plan(const isa_params* p, const void* q, const void* k, const voi
     return s;
   const PlanLayout L = make_layout(d);
   if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
-  if ((s = ensure_init()) != ISA_OK) return s;
+  if ((s = ensure_init()) != ISA_OK || (s = bind_device_of(q, "q")) != ISA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const PlanPtrs pp = make_ptrs(L, ws);
   cudaError_t e = cudaMemsetAsync(pp.status, 0, 256, st);
@@ -253,23 +276,10 @@ isa_status isa_plan(const isa_params* p, const void* q, const void* k, const voi
   return ISA_OK;
 }
 
-static isa_status run_attention(const Dims& d, int mode, const void* q, const void* k, const void* v,
-                                const PlanPtrs* pp, void* out, float* lse, int32_t* status, cudaStream_t st) {
-  isa_status s;
+// Sizes, plan pointers and work-list counts of the attention kernels (mode 0:
+// ISA items from the plan; mode 1: dense items).
+static AttnArgs attn_args(const Dims& d, int mode, const PlanPtrs* pp) {
   const int R = mode == 1 ? 64 : d.b;
-  CUtensorMap maps[5];
-  const uint64_t rows = (uint64_t)d.BH * d.L;
-  if ((s = make_map(&maps[0], q, rows, d.D, R, "q")) != ISA_OK) return s;
-  if ((s = make_map(&maps[1], k, rows, d.D, R, "k")) != ISA_OK) return s;
-  if ((s = make_map(&maps[2], v, rows, d.D, R, "v")) != ISA_OK) return s;
-  if (pp) {
-    const uint64_t prow = (uint64_t)d.BH * d.T_kv_pad;
-    if ((s = make_map(&maps[3], pp->Kp, prow, d.D, R, "Kp")) != ISA_OK) return s;
-    if ((s = make_map(&maps[4], pp->Vp, prow, d.D, R, "Vp")) != ISA_OK) return s;
-  } else {
-    maps[3] = maps[1];
-    maps[4] = maps[2];
-  }
   AttnArgs a{};
   a.BH = d.BH;
   a.L = d.L;
@@ -300,16 +310,52 @@ static isa_status run_attention(const Dims& d, int mode, const void* q, const vo
     a.bits = pp->bits;
     a.ctx_sel = pp->ctx_sel;
   }
+  a.timeout_ns = g_timeout_ns;
+  a.inject = g_inject;
+  return a;
+}
+
+static isa_status run_attention(const Dims& d, int mode, const void* q, const void* k, const void* v,
+                                const PlanPtrs* pp, void* out, float* lse, int32_t* status, cudaStream_t st) {
+  isa_status s;
+  const int R = mode == 1 ? 64 : d.b;
+  CUtensorMap maps[5];
+  const uint64_t rows = (uint64_t)d.BH * d.L;
+  if ((s = make_map(&maps[0], q, rows, d.D, R, "q")) != ISA_OK) return s;
+  if ((s = make_map(&maps[1], k, rows, d.D, R, "k")) != ISA_OK) return s;
+  if ((s = make_map(&maps[2], v, rows, d.D, R, "v")) != ISA_OK) return s;
+  if (pp) {
+    const uint64_t prow = (uint64_t)d.BH * d.T_kv_pad;
+    if ((s = make_map(&maps[3], pp->Kp, prow, d.D, R, "Kp")) != ISA_OK) return s;
+    if ((s = make_map(&maps[4], pp->Vp, prow, d.D, R, "Vp")) != ISA_OK) return s;
+  } else {
+    maps[3] = maps[1];
+    maps[4] = maps[2];
+  }
+  AttnArgs a = attn_args(d, mode, pp);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
   a.status = status;
-  a.timeout_ns = g_timeout_ns;
-  a.inject = g_inject;
   if (a.total_items == 0) return ISA_OK;
   const int grid = std::min(sm_count(), a.total_items);
   cudaError_t e = launch_attention(d.D, R, maps, a, grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ISA_OK;
+}
+
+// Byte offsets of the backward workspace: per query row (lse2, Delta), then
+// the fp32 gradients of the pooled keys and values.
+struct BwdLayout {
+  size_t dl, dKc, dVc, total;
+};
+
+static BwdLayout bwd_layout(const Dims& d) {
+  BwdLayout L{};
+  L.dl = 0;
+  L.dKc = align256((size_t)d.BH * d.L * 8);
+  L.dVc = L.dKc + align256((size_t)d.BH * d.T_kv_pad * d.D * 4);
+  L.total = L.dVc + align256((size_t)d.BH * d.T_kv_pad * d.D * 4);
+  return L;
 }
 
 isa_status isa_forward(const isa_params* p, const void* q, const void* k, const void* v, const void* ws,
@@ -324,7 +370,7 @@ isa_status isa_forward(const isa_params* p, const void* q, const void* k, const 
   if (lse && (s = check_ptr(lse, "lse", 4)) != ISA_OK) return s;
   const PlanLayout L = make_layout(d);
   if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
-  if ((s = ensure_init()) != ISA_OK) return s;
+  if ((s = ensure_init()) != ISA_OK || (s = bind_device_of(q, "q")) != ISA_OK) return s;
   const PlanPtrs pp = make_ptrs(L, const_cast<void*>(ws));
   return run_attention(d, 0, q, k, v, &pp, out, lse, pp.status, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -339,13 +385,70 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
     return s;
   if (lse && (s = check_ptr(lse, "lse", 4)) != ISA_OK) return s;
   if (status && (s = check_ptr(status, "status", 4)) != ISA_OK) return s;
-  if ((s = ensure_init()) != ISA_OK) return s;
+  if ((s = ensure_init()) != ISA_OK || (s = bind_device_of(q, "q")) != ISA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (status) {
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
   }
   return run_attention(d, 1, q, k, v, nullptr, out, lse, status, st);
+}
+
+isa_status isa_backward_workspace_size(const isa_params* p, size_t* bytes) {
+  if (!bytes) return fail(ISA_ERR_INVALID_ARG, "bytes is NULL");
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  *bytes = bwd_layout(d).total;
+  return ISA_OK;
+}
+
+isa_status isa_backward(const isa_params* p, const void* q, const void* k, const void* v, const void* ws,
+                        size_t ws_bytes, const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                        void* dv, void* bws, size_t bws_bytes, void* stream) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if ((s = check_ptr(q, "q", 16)) != ISA_OK || (s = check_ptr(k, "k", 16)) != ISA_OK ||
+      (s = check_ptr(v, "v", 16)) != ISA_OK || (s = check_ptr(ws, "workspace", 256)) != ISA_OK ||
+      (s = check_ptr(out, "out", 16)) != ISA_OK || (s = check_ptr(lse, "lse", 4)) != ISA_OK ||
+      (s = check_ptr(dout, "dout", 16)) != ISA_OK || (s = check_ptr(dq, "dq", 16)) != ISA_OK ||
+      (s = check_ptr(dk, "dk", 16)) != ISA_OK || (s = check_ptr(dv, "dv", 16)) != ISA_OK ||
+      (s = check_ptr(bws, "backward workspace", 256)) != ISA_OK)
+    return s;
+  const PlanLayout L = make_layout(d);
+  if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  const BwdLayout BL = bwd_layout(d);
+  if (bws_bytes < BL.total)
+    return fail(ISA_ERR_WORKSPACE, "backward workspace has %zu bytes, needs %zu", bws_bytes, BL.total);
+  if ((s = ensure_init()) != ISA_OK || (s = bind_device_of(q, "q")) != ISA_OK) return s;
+  const PlanPtrs pp = make_ptrs(L, const_cast<void*>(ws));
+  CUtensorMap maps[6];
+  const uint64_t rows = (uint64_t)d.BH * d.L, prow = (uint64_t)d.BH * d.T_kv_pad;
+  if ((s = make_map(&maps[0], q, rows, d.D, d.b, "q")) != ISA_OK) return s;
+  if ((s = make_map(&maps[1], k, rows, d.D, d.b, "k")) != ISA_OK) return s;
+  if ((s = make_map(&maps[2], v, rows, d.D, d.b, "v")) != ISA_OK) return s;
+  if ((s = make_map(&maps[3], pp.Kp, prow, d.D, d.b, "Kp")) != ISA_OK) return s;
+  if ((s = make_map(&maps[4], pp.Vp, prow, d.D, d.b, "Vp")) != ISA_OK) return s;
+  if ((s = make_map(&maps[5], dout, rows, d.D, d.b, "dout")) != ISA_OK) return s;
+  BwdArgs b{};
+  b.a = attn_args(d, 0, &pp);
+  b.a.status = pp.status;
+  b.o = static_cast<const __nv_bfloat16*>(out);
+  b.dout = static_cast<const __nv_bfloat16*>(dout);
+  b.lse = lse;
+  char* w = static_cast<char*>(bws);
+  b.dl = reinterpret_cast<float2*>(w + BL.dl);
+  b.dKc = reinterpret_cast<float*>(w + BL.dKc);
+  b.dVc = reinterpret_cast<float*>(w + BL.dVc);
+  b.dq = static_cast<__nv_bfloat16*>(dq);
+  b.dk = static_cast<__nv_bfloat16*>(dk);
+  b.dv = static_cast<__nv_bfloat16*>(dv);
+  b.scale = d.scale;
+  b.has_pooled = (d.n_flat > 0 && d.n_exact < d.T_kv) ? 1 : 0;
+  cudaError_t e = launch_backward(d, maps, b, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return ISA_OK;
 }
 
 isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes) {
@@ -369,6 +472,7 @@ isa_status isa_rope(const isa_params* p, float base, const void* q, const void* 
     return s;
   const size_t need = rope_table_bytes(d);
   if (ws_bytes < need) return fail(ISA_ERR_WORKSPACE, "rope workspace has %zu bytes, needs %zu", ws_bytes, need);
+  if ((s = bind_device_of(q, "q")) != ISA_OK) return s;
   cudaError_t e = launch_rope(d, (double)base, q, k, q_out, k_out, ws, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rope launch");
   return ISA_OK;

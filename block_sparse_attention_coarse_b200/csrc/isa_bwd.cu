@@ -1,0 +1,939 @@
+// Backward of the ISA sparse attention for sm_100a: gradients of steps
+// (4)-(6) of "Method steps in detail" (paper.rainbus.top summary card of
+// "LIVEditor-14B: Lightning Unified Video Editing via In-Context Sparse
+// Attention") with respect to Q, K and V, with the plan held fixed.  The
+// pages state that the method has a differentiable forward + backward
+// implementation and is trained end to end ("Core method", innovation (c))
+// without giving formulas; the gradients here are those of the forward as
+// computed: the plan's index sets carry no gradient, and the pooled means
+// Kc_j, Vc_j of the flat path pass their gradient to every token of block j
+// with weight 1/n_j.
+//
+// With P the softmax weights of a query row over its columns (exact key
+// tokens and, for flat rows, pooled keys with log-weight ln n_j), dP = dO V^T
+// and Delta = rowsum(dO * O):
+//   dS = P * (dP - Delta),  dQ = s dS K,  dK = s dS^T Q,  dV = P^T dO.
+//
+// Launches, in stream order:
+//   bwd_prep_kernel        Delta and lse*log2(e) per query row (HBM-bound)
+//   bwd_zero_unkept_kernel dK = dV = 0 for context blocks the pre-selection dropped
+//   bwd_kv_kernel (pooled) key/value-stationary over the head's pooled rows:
+//                          dKc_j, dVc_j (fp32) from every flat block
+//   bwd_kv_kernel (kept)   key/value-stationary over the kept blocks: dK, dV
+//                          from the sharp blocks and the flat blocks that
+//                          attend the block exactly, plus dKc_j/n_j, dVc_j/n_j
+//   bwd_q_kernel           query-stationary over the forward's work items: dQ
+// P is recomputed from the forward's lse, so no attention matrix is stored.
+#include <algorithm>
+
+#include "isa_common.cuh"
+#include "isa_items.cuh"
+
+namespace isa {
+
+namespace bwd {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// per-row preparation
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
+  const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 fx = __bfloat1622float2(x[i]), fy = __bfloat1622float2(y[i]);
+    acc = fmaf(fx.x, fy.x, acc);
+    acc = fmaf(fx.y, fy.y, acc);
+  }
+  return acc;
+}
+
+// dl[r] = (lse[r] * log2 e, sum_d dout[r, d] * o[r, d]); D/8 lanes per row,
+// grid-stride over the rows (the loop bound is warp-uniform).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
+                                                       const float* __restrict__ lse, float2* __restrict__ dl,
+                                                       size_t rows) {
+  constexpr int LPR = D / 8;
+  constexpr int RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const size_t warp = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const size_t nwarps = ((size_t)gridDim.x * blockDim.x) >> 5;
+  for (size_t r0 = warp * RPW; r0 < rows; r0 += nwarps * RPW) {
+    const size_t r = r0 + lane / LPR;
+    float acc = 0.f;
+    if (r < rows) acc = dot_bf16x8(o[r * LPR + lane % LPR], dout[r * LPR + lane % LPR]);
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+    if (r < rows && lane % LPR == 0) dl[r] = make_float2(lse[r] * kLog2e, acc);
+  }
+}
+
+// dK and dV rows of context block blockIdx.y of head blockIdx.x are zero when
+// the pre-selection dropped the block (it takes part in neither path).
+__global__ void __launch_bounds__(128) bwd_zero_unkept_kernel(const int* __restrict__ ctx_sel, int K_sel, int L,
+                                                              int L_src, int L_ctx, int b, int D, uint4* dk, uint4* dv) {
+  const int bh = blockIdx.x, c = blockIdx.y;
+  const int* sel = ctx_sel + (size_t)bh * K_sel;
+  int lo = 0, hi = K_sel;   // ctx_sel is ascending
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (sel[mid] < c) lo = mid + 1;
+    else hi = mid;
+  }
+  if (lo < K_sel && sel[lo] == c) return;
+  const int s = c * b;
+  const int n = min(b, L_ctx - s);
+  const size_t first = ((size_t)bh * L + L_src + s) * (D / 8);
+  const size_t cnt = (size_t)n * (D / 8);
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (size_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+    dk[first + i] = z;
+    dv[first + i] = z;
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// key/value-stationary kernel: dK, dV
+// ---------------------------------------------------------------------------
+// An item is one 128-row key/value tile of one head and stays in shared
+// memory while 64-row query steps stream past it:
+//   kept launch   : rows = G = 128/R consecutive kept blocks (kept positions
+//                   tile*G ..); steps = every sharp block, then the flat
+//                   blocks whose exact list holds one of the tile's blocks
+//                   (rows of the other blocks masked per query block)
+//   pooled launch : rows = 128 consecutive pooled kept blocks (Kp/Vp rows);
+//                   steps = every flat block, with the flat block's own exact
+//                   blocks masked out; log-weight log2(n_j) per row
+// Per step (TMEM lane = key/value row):
+//   S^T = K Q^T, dP^T = V dO^T         (SS, M=128, N=64, K=D)
+//   P^T = 2^(S^T s log2e + w_j - lse2), dS^T = P^T (dP^T - Delta)   (softmax warps)
+//   dV += P^T dO, dK += dS^T Q         (TS: P^T / dS^T read as bf16 from TMEM)
+// Roles (320 threads, one CTA per SM): warp 0 lane 0 TMA producer (the tile,
+// the query/dO steps and their metadata), warp 1 MMA issuer (converged, one
+// elected lane), warps 2..9: warp w owns TMEM lanes 32*(w%4).. and query
+// columns 32*((w-2)/4).. of each step, and writes the epilogue.
+constexpr int kKvThreads = 320;
+constexpr int kNSQ = 3;           // query/dO step stages
+constexpr uint32_t kTST = 0;      // S^T then P^T (bf16): two buffers of 64 columns
+constexpr uint32_t kTDP = 128;    // dP^T then dS^T (bf16): two buffers of 64 columns
+constexpr uint32_t kTDV = 256;    // dV accumulator (D columns); dK at kTDV + D
+
+template <int D, int R>
+struct KvCfg {
+  static constexpr int G = 128 / R;               // kept blocks per tile
+  static constexpr int GQ = 64 / R;               // query blocks per step
+  static constexpr int NCH = D / 64;              // 64-column chunks of a row
+  static constexpr uint32_t CHUNK = 128 * 128;    // 128 rows x 128 bytes
+  static constexpr uint32_t QCHUNK = 64 * 128;    // 64 rows x 128 bytes
+  static constexpr uint32_t TILE = 128 * D * 2;
+  static constexpr uint32_t QTILE = 64 * D * 2;
+  static constexpr uint32_t BOX = R * 128;        // one TMA box
+  static constexpr uint32_t K_OFF = 0;
+  static constexpr uint32_t V_OFF = TILE;
+  static constexpr uint32_t Q_OFF = 2 * TILE;
+  static constexpr uint32_t DO_OFF = Q_OFF + kNSQ * QTILE;
+  static constexpr uint32_t SMEM_USED = DO_OFF + kNSQ * QTILE + 1024;
+  // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits on an SM
+  static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr uint32_t ID_T = idesc_bf16_f32(128, 64, 0);
+  static constexpr uint32_t ID_A = idesc_bf16_f32(128, D, 1);
+};
+
+struct StepMeta {
+  int start[2], cnt[2];   // token start and valid rows of the step's query blocks
+  uint32_t m[2][4];       // tile rows each query block attends (bit r of m[g][r/32])
+  int last;               // last step of the item
+};
+
+__device__ __forceinline__ void clear_meta(StepMeta& m) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    m.start[g] = 0;
+    m.cnt[g] = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) m.m[g][w] = 0u;
+  }
+  m.last = 0;
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(kKvThreads, 1)
+    bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                  const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdArgs b) {
+  using C = KvCfg<D, R>;
+  constexpr int G = C::G, GQ = C::GQ;
+  const AttnArgs& a = b.a;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t kv_full, kv_empty, q_full[kNSQ], q_empty[kNSQ], sd_full[2], ds_full[2];
+  __shared__ __align__(8) uint64_t acc_ready, acc_free, drain_bar;
+  __shared__ StepMeta meta[kNSQ];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const bool pooled = b.kv_pooled != 0;
+
+  if (tid == 0) {
+    mbar_init(&kv_full, 1);
+    mbar_init(&kv_empty, 1);
+    for (int i = 0; i < kNSQ; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sd_full[i], 1);
+      mbar_init(&ds_full[i], 256);
+    }
+    mbar_init(&acc_ready, 1);
+    mbar_init(&acc_free, 256);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(pooled ? &tm_kp : &tm_k);
+    tma_prefetch_desc(pooled ? &tm_vp : &tm_v);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const WaitCtl wc{&abort_flag, a.status, a.timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      int kv_cnt = 0, qcnt[kNSQ];
+      for (int i = 0; i < kNSQ; ++i) qcnt[i] = 0;
+      int u = 0, n = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
+        const int bh = it / b.kv_tiles, tile = it % b.kv_tiles;
+        if (n >= 1 && !mbar_wait(&kv_empty, (n - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&kv_full, 2 * C::TILE);
+        ++kv_cnt;
+        for (int g = 0; g < G; ++g) {
+          int row;
+          if (pooled) {
+            row = bh * a.T_kv_pad + tile * 128 + g * R;
+          } else {
+            const int kk = tile * G + g;
+            row = bh * a.L;
+            if (kk < a.T_kv) row += block_span(a.kept[(size_t)bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src).x;
+          }
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_2d(sgen + C::K_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_kp : &tm_k, c * 64, row, &kv_full);
+            tma_load_2d(sgen + C::V_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_vp : &tm_v, c * 64, row, &kv_full);
+          }
+        }
+        // Steps are published one behind, so that the last one can be marked.
+        StepMeta pend, grp;
+        bool have = false;
+        int ng = 0;
+        auto emit = [&](const StepMeta& m, int last) -> bool {
+          const int s = u % kNSQ;
+          if (u >= kNSQ && !mbar_wait(&q_empty[s], ((u / kNSQ) - 1) & 1, wc)) return false;
+          meta[s] = m;
+          meta[s].last = last;   // published by the arrive below (release), read after q_full (acquire)
+          mbar_arrive_expect_tx(&q_full[s], 2 * C::QTILE);
+          ++qcnt[s];
+          for (int g = 0; g < GQ; ++g) {
+            const int row = bh * a.L + (m.cnt[g] > 0 ? m.start[g] : 0);
+            for (int c = 0; c < C::NCH; ++c) {
+              tma_load_2d(sgen + C::Q_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_q, c * 64, row,
+                          &q_full[s]);
+              tma_load_2d(sgen + C::DO_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_do, c * 64, row,
+                          &q_full[s]);
+            }
+          }
+          ++u;
+          return true;
+        };
+        auto push = [&](const StepMeta& m) -> bool {
+          const bool r = have ? emit(pend, 0) : true;
+          pend = m;
+          have = true;
+          return r;
+        };
+        if (!pooled) {
+          // sharp blocks attend every kept block: all rows of the tile
+          for (int s0 = 0; ok && s0 < a.n_sharp; s0 += GQ) {
+            StepMeta m;
+            clear_meta(m);
+            for (int g = 0; g < GQ; ++g) {
+              if (s0 + g >= a.n_sharp) break;
+              const int2 sp = block_span(a.sharp[(size_t)bh * a.n_sharp + s0 + g], a.L_src, a.L_ctx, a.b, a.T_src);
+              m.start[g] = sp.x;
+              m.cnt[g] = sp.y;
+              for (int w = 0; w < 4; ++w) m.m[g][w] = 0xFFFFFFFFu;
+            }
+            ok = push(m);
+          }
+        }
+        clear_meta(grp);
+        for (int f = 0; ok && f < a.n_flat; ++f) {
+          const uint32_t* fb = a.bits + ((size_t)bh * a.n_flat + f) * a.words;
+          uint32_t mw[4];
+          bool any = false;
+          if (pooled) {
+            // pooled rows tile*128 + r, minus the flat block's exact blocks
+            for (int w = 0; w < 4; ++w) {
+              const int wi = tile * 4 + w;
+              const int rem = a.T_kv - (tile * 128 + 32 * w);
+              const uint32_t range = rem >= 32 ? 0xFFFFFFFFu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
+              mw[w] = range & ~(wi < a.words ? fb[wi] : 0u);
+              any = any || mw[w] != 0u;
+            }
+          } else {
+            // exact blocks among kept positions tile*G .. tile*G+G-1 (one word)
+            const int k0 = tile * G;
+            const uint32_t gm = (fb[k0 >> 5] >> (k0 & 31)) & ((1u << G) - 1u);
+            any = gm != 0u;
+            for (int w = 0; w < 4; ++w) mw[w] = ((gm >> ((32 * w) / R)) & 1u) ? 0xFFFFFFFFu : 0u;
+          }
+          if (!any) continue;
+          const int2 sp = block_span(a.flat[(size_t)bh * a.n_flat + f], a.L_src, a.L_ctx, a.b, a.T_src);
+          grp.start[ng] = sp.x;
+          grp.cnt[ng] = sp.y;
+          for (int w = 0; w < 4; ++w) grp.m[ng][w] = mw[w];
+          if (++ng == GQ) {
+            ok = push(grp);
+            clear_meta(grp);
+            ng = 0;
+          }
+        }
+        if (ok && ng > 0) ok = push(grp);
+        if (ok && !have) {
+          clear_meta(pend);   // no query attends the tile: one empty step writes zeros
+          have = true;
+        }
+        if (ok) ok = emit(pend, 1);
+      }
+      // let every copy in flight land before the CTA can exit
+      if (kv_cnt) mbar_wait_drain(&kv_full, (kv_cnt - 1) & 1, a.timeout_ns);
+      for (int i = 0; i < kNSQ; ++i)
+        if (qcnt[i]) mbar_wait_drain(&q_full[i], (qcnt[i] - 1) & 1, a.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool issued = false, ok = true;
+    int u = 0, n = 0;
+    const uint64_t kdesc = smem_desc_sw128(sbase + C::K_OFF, 16, 1024);
+    const uint64_t vdesc = smem_desc_sw128(sbase + C::V_OFF, 16, 1024);
+    // S^T and dP^T of step uu into buffer uu % 2
+    auto issue_t = [&](int uu) -> bool {
+      const int s = uu % kNSQ;
+      if (!warp_wait(&q_full[s], (uu / kNSQ) & 1, wc)) return false;
+      tc_fence_after();
+      const uint64_t qd = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, 16, 1024);
+      const uint64_t dd = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, 16, 1024);
+      const uint32_t col = (uu & 1) * 64;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTST + col, kdesc + oa, qd + ob, C::ID_T, ks > 0);
+      }
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTDP + col, vdesc + oa, dd + ob, C::ID_T, ks > 0);
+      }
+      issued = true;
+      tc_commit_elect(&sd_full[uu & 1]);
+      return true;
+    };
+    for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
+      if (!warp_wait(&kv_full, n & 1, wc)) break;
+      tc_fence_after();
+      if (!(ok = issue_t(u))) break;
+      for (bool first = true;; first = false) {
+        const int s = u % kNSQ;
+        const int last = meta[s].last;
+        // the next step's S^T, dP^T go to the other buffers while the softmax
+        // warps work on this one
+        if (!last && !(ok = issue_t(u + 1))) break;
+        if (!warp_wait(&ds_full[u & 1], (u >> 1) & 1, wc) ||
+            (first && n > 0 && !warp_wait(&acc_free, (n - 1) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t qmn = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, C::QCHUNK, 1024);
+        const uint64_t dmn = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, C::QCHUNK, 1024);
+        const uint32_t col = (u & 1) * 64;
+        // packed bf16 P^T / dS^T: warp half h holds query columns 32h..32h+31
+        // in its buffer's columns 32h..32h+15
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts_elect(tmem + kTDV, tmem + kTST + col + (ks >> 1) * 32 + (ks & 1) * 8,
+                       dmn + (uint64_t)(ks * 2048 >> 4), C::ID_A, (!first || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts_elect(tmem + kTDV + D, tmem + kTDP + col + (ks >> 1) * 32 + (ks & 1) * 8,
+                       qmn + (uint64_t)(ks * 2048 >> 4), C::ID_A, (!first || ks > 0) ? 1u : 0u);
+        tc_commit_elect(&q_empty[s]);
+        ++u;
+        if (last) break;
+      }
+      if (!ok) break;
+      tc_commit_elect(&acc_ready);
+      tc_commit_elect(&kv_empty);
+    }
+    if (issued) {
+      tc_commit_elect(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0, a.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3, hw = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;                      // tile row = TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int gq = (R == 32) ? hw : 0;                      // this thread's query block of a step
+    const int coff = (R == 32) ? 0 : 32 * hw;               // its first column within that block
+    const float sl2 = a.sl2;
+    constexpr int DH = D / 2;
+    int u = 0, n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
+      const int bh = it / b.kv_tiles, tile = it % b.kv_tiles;
+      bool row_valid = false;
+      int tok = 0, kk = 0, nj = 1;
+      float bias = 0.f;
+      if (pooled) {
+        kk = tile * 128 + r;
+        row_valid = kk < a.T_kv;
+        if (row_valid) {
+          nj = block_span(a.kept[(size_t)bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src).y;
+          bias = __log2f((float)nj);
+        }
+      } else {
+        kk = tile * G + r / R;
+        if (kk < a.T_kv) {
+          const int2 sp = block_span(a.kept[(size_t)bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src);
+          nj = sp.y;
+          row_valid = (r % R) < sp.y;
+          tok = sp.x + r % R;
+        }
+      }
+      const float2* dlh = b.dl + (size_t)bh * a.L;
+      for (;;) {
+        const int s = u % kNSQ, buf = u & 1;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sd_full[buf], (u >> 1) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int st0 = meta[s].start[gq], cn = meta[s].cnt[gq], last = meta[s].last;
+        const bool on = row_valid && ((meta[s].m[gq][r >> 5] >> (r & 31)) & 1u);
+        // lane c fetches (lse2, Delta) of column coff + c; shared by shuffles
+        const int c = coff + lane;
+        const float2 mine = c < cn ? dlh[st0 + c] : make_float2(INFINITY, 0.f);
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tl + kTST + buf * 64 + 32 * hw, sv);
+        tmem_ld32(tl + kTDP + buf * 64 + 32 * hw, dp);
+        tmem_wait_ld();
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float l0 = __shfl_sync(0xFFFFFFFFu, mine.x, e), l1 = __shfl_sync(0xFFFFFFFFu, mine.x, e + 1);
+          const float d0 = __shfl_sync(0xFFFFFFFFu, mine.y, e), d1 = __shfl_sync(0xFFFFFFFFu, mine.y, e + 1);
+          float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, bias - l0));
+          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, bias - l1));
+          if (!on) p0 = p1 = 0.f;
+          const float g0 = p0 * (__uint_as_float(dp[e]) - d0);
+          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - d1);
+          pp[e >> 1] = pack_bf16x2(p0, p1);
+          pd[e >> 1] = pack_bf16x2(g0, g1);
+        }
+        tmem_st16(tl + kTST + buf * 64 + 32 * hw, pp);
+        tmem_st16(tl + kTDP + buf * 64 + 32 * hw, pd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ds_full[buf]);
+        ++u;
+        if (last) break;
+      }
+      if (!ok) break;
+      // epilogue: this thread's DH columns of dV and dK for tile row r
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_ready, n & 1, wc))) break;
+      tc_fence_after();
+      uint32_t gv[DH / 32][32], gk[DH / 32][32];
+#pragma unroll
+      for (int c0 = 0; c0 < DH / 32; ++c0) {
+        tmem_ld32(tl + kTDV + hw * DH + 32 * c0, gv[c0]);
+        tmem_ld32(tl + kTDV + D + hw * DH + 32 * c0, gk[c0]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&acc_free);
+      if (!row_valid) continue;
+      const float sc = b.scale;
+      if (pooled) {
+        float4* kd = reinterpret_cast<float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
+        float4* vd = reinterpret_cast<float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
+#pragma unroll
+        for (int e = 0; e < DH; e += 4) {
+          const uint32_t* k4 = &gk[e >> 5][e & 31];
+          const uint32_t* v4 = &gv[e >> 5][e & 31];
+          kd[e >> 2] = make_float4(sc * __uint_as_float(k4[0]), sc * __uint_as_float(k4[1]),
+                                   sc * __uint_as_float(k4[2]), sc * __uint_as_float(k4[3]));
+          vd[e >> 2] = make_float4(__uint_as_float(v4[0]), __uint_as_float(v4[1]), __uint_as_float(v4[2]),
+                                   __uint_as_float(v4[3]));
+        }
+      } else {
+        // this block's share of its pooled-mean gradient: dKc_j / n_j, dVc_j / n_j
+        const float inv = 1.f / (float)nj;
+        const float4* kc = reinterpret_cast<const float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
+        const float4* vc = reinterpret_cast<const float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
+        uint4* kd = reinterpret_cast<uint4*>(b.dk + ((size_t)bh * a.L + tok) * D + hw * DH);
+        uint4* vd = reinterpret_cast<uint4*>(b.dv + ((size_t)bh * a.L + tok) * D + hw * DH);
+#pragma unroll
+        for (int e = 0; e < DH; e += 8) {
+          float xk[8], xv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            xk[i] = sc * __uint_as_float(gk[(e + i) >> 5][(e + i) & 31]);
+            xv[i] = __uint_as_float(gv[(e + i) >> 5][(e + i) & 31]);
+          }
+          if (b.has_pooled) {
+            const float4 k0 = kc[e >> 2], k1 = kc[(e >> 2) + 1], v0 = vc[e >> 2], v1 = vc[(e >> 2) + 1];
+            xk[0] = fmaf(k0.x, inv, xk[0]); xk[1] = fmaf(k0.y, inv, xk[1]);
+            xk[2] = fmaf(k0.z, inv, xk[2]); xk[3] = fmaf(k0.w, inv, xk[3]);
+            xk[4] = fmaf(k1.x, inv, xk[4]); xk[5] = fmaf(k1.y, inv, xk[5]);
+            xk[6] = fmaf(k1.z, inv, xk[6]); xk[7] = fmaf(k1.w, inv, xk[7]);
+            xv[0] = fmaf(v0.x, inv, xv[0]); xv[1] = fmaf(v0.y, inv, xv[1]);
+            xv[2] = fmaf(v0.z, inv, xv[2]); xv[3] = fmaf(v0.w, inv, xv[3]);
+            xv[4] = fmaf(v1.x, inv, xv[4]); xv[5] = fmaf(v1.y, inv, xv[5]);
+            xv[6] = fmaf(v1.z, inv, xv[6]); xv[7] = fmaf(v1.w, inv, xv[7]);
+          }
+          kd[e >> 3] = make_uint4(pack_bf16x2(xk[0], xk[1]), pack_bf16x2(xk[2], xk[3]), pack_bf16x2(xk[4], xk[5]),
+                                  pack_bf16x2(xk[6], xk[7]));
+          vd[e >> 3] = make_uint4(pack_bf16x2(xv[0], xv[1]), pack_bf16x2(xv[2], xv[3]), pack_bf16x2(xv[4], xv[5]),
+                                  pack_bf16x2(xv[6], xv[7]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// query-stationary kernel: dQ
+// ---------------------------------------------------------------------------
+// The forward's work items (G query blocks of one head, the same KV tiles
+// and column masks).  Per tile t:
+//   S = Q K_t^T, dP = dO V_t^T          (SS, M=128, N=128, K=D)
+//   P = 2^(S s log2e + w - lse2), dS = P (dP - Delta)   (softmax warps, bf16 dS into TMEM)
+//   dQ += dS K_t                        (TS, K_t read as the MN-major operand)
+// Roles as in the forward (352 threads): warp 0 lane 0 loads Q, dO and the
+// K tiles, warp 10 lane 0 the V tiles, warp 1 issues the MMAs, warps 2..9
+// hold 16 query rows each (a row split between threads t and t+16).
+// TMEM: S/dS buffers at 0 and 128 (tile t in t % 2), dP at 256 (one buffer,
+// released as soon as the softmax warps have loaded it), dQ at 384.
+constexpr int kQThreads = 352;
+constexpr int kQNSK = 3;
+constexpr int kQNSV = 2;
+constexpr uint32_t kTS = 0;
+constexpr uint32_t kTP = 256;
+constexpr uint32_t kTQ = 384;
+
+template <int D, int R>
+struct QCfg {
+  static constexpr int G = 128 / R;
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t CHUNK = 128 * 128;
+  static constexpr uint32_t TILE = 128 * D * 2;
+  static constexpr uint32_t BOX = R * 128;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t DO_OFF = TILE;
+  static constexpr uint32_t K_OFF = 2 * TILE;
+  static constexpr uint32_t V_OFF = K_OFF + kQNSK * TILE;
+  static constexpr uint32_t SMEM_USED = V_OFF + kQNSV * TILE + 1024;
+  static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0);
+  static constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1);
+};
+
+template <int D, int R>
+__global__ void __launch_bounds__(kQThreads, 1)
+    bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                 const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_do,
+                 const BwdArgs b) {
+  using C = QCfg<D, R>;
+  constexpr int G = C::G;
+  const AttnArgs& a = b.a;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full, q_empty, k_full[kQNSK], k_empty[kQNSK], v_full[kQNSV], v_empty[kQNSV];
+  __shared__ __align__(8) uint64_t sd_full[2], dp_free, ds_full[2], dq_ready, dq_free, drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+
+  if (tid == 0) {
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
+    for (int i = 0; i < kQNSK; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kQNSV; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sd_full[i], 1);
+      mbar_init(&ds_full[i], 256);
+    }
+    mbar_init(&dp_free, 256);
+    mbar_init(&dq_ready, 1);
+    mbar_init(&dq_free, 256);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_kp);
+    tma_prefetch_desc(&tm_vp);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const WaitCtl wc{&abort_flag, a.status, a.timeout_ns};
+
+  if ((warp == 0 || warp == 10) && lane == 0) {
+    // ------------------------------------------------------------ producers
+    const bool kside = warp == 0;
+    int q_cnt = 0, cnt[kQNSK > kQNSV ? kQNSK : kQNSV];
+    const int ns = kside ? kQNSK : kQNSV;
+    for (int i = 0; i < ns; ++i) cnt[i] = 0;
+    uint64_t* full = kside ? k_full : v_full;
+    uint64_t* empty = kside ? k_empty : v_empty;
+    const uint32_t off = kside ? C::K_OFF : C::V_OFF;
+    int n = 0, t = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      if (kside) {
+        if (n >= 1 && !mbar_wait(&q_empty, (n - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&q_full, 2 * C::TILE);
+        ++q_cnt;
+        for (int g = 0; g < G; ++g) {
+          const int2 sp = q_span<R>(a, I, g);
+          const int row = I.bh * a.L + (sp.y > 0 ? sp.x : 0);
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_2d(sgen + C::Q_OFF + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full);
+            tma_load_2d(sgen + C::DO_OFF + c * C::CHUNK + g * C::BOX, &tm_do, c * 64, row, &q_full);
+          }
+        }
+      }
+      for (int j = 0; j < I.ntiles; ++j, ++t) {
+        const int s = t % ns;
+        if (t >= ns && !mbar_wait(&empty[s], ((t / ns) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        int rows[G];
+        bool pooled = false;
+        for (int g = 0; g < G; ++g) {
+          const int3 sp = kv_span<R, G>(a, I, j, g);
+          pooled = sp.z != 0;
+          rows[g] = pooled ? I.bh * a.T_kv_pad + sp.x : I.bh * a.L + (sp.y > 0 ? sp.x : 0);
+        }
+        const CUtensorMap* m = kside ? (pooled ? &tm_kp : &tm_k) : (pooled ? &tm_vp : &tm_v);
+        mbar_arrive_expect_tx(&full[s], C::TILE);
+        ++cnt[s];
+        for (int g = 0; g < G; ++g)
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_2d(sgen + off + s * C::TILE + c * C::CHUNK + g * C::BOX, m, c * 64, rows[g], &full[s]);
+      }
+    }
+    if (q_cnt) mbar_wait_drain(&q_full, (q_cnt - 1) & 1, a.timeout_ns);
+    for (int i = 0; i < ns; ++i)
+      if (cnt[i]) mbar_wait_drain(&full[i], (cnt[i] - 1) & 1, a.timeout_ns);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool issued = false, ok = true;
+    int n = 0, t0 = 0;
+    const uint64_t qdesc = smem_desc_sw128(sbase + C::Q_OFF, 16, 1024);
+    const uint64_t odesc = smem_desc_sw128(sbase + C::DO_OFF, 16, 1024);
+    // S_t = Q K_t^T into buffer t % 2
+    auto issue_s = [&](int t) -> bool {
+      const int s = t % kQNSK;
+      if (!warp_wait(&k_full[s], (t / kQNSK) & 1, wc)) return false;
+      tc_fence_after();
+      const uint64_t kdesc = smem_desc_sw128(sbase + C::K_OFF + s * C::TILE, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTS + (t & 1) * 128, qdesc + o, kdesc + o, C::ID_S, ks > 0);
+      }
+      issued = true;
+      return true;
+    };
+    // dP_t = dO V_t^T once the softmax warps have loaded dP_{t-1}; then S_t
+    // and dP_t are announced together
+    auto issue_dp = [&](int t) -> bool {
+      const int s = t % kQNSV;
+      if ((t > 0 && !warp_wait(&dp_free, (t - 1) & 1, wc)) || !warp_wait(&v_full[s], (t / kQNSV) & 1, wc))
+        return false;
+      tc_fence_after();
+      const uint64_t vdesc = smem_desc_sw128(sbase + C::V_OFF + s * C::TILE, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTP, odesc + o, vdesc + o, C::ID_S, ks > 0);
+      }
+      tc_commit_elect(&v_empty[s]);
+      tc_commit_elect(&sd_full[t & 1]);
+      return true;
+    };
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      const int nt = I.ntiles;
+      if (!warp_wait(&q_full, n & 1, wc)) break;
+      tc_fence_after();
+      if (!(ok = issue_s(t0) && issue_dp(t0))) break;
+      if (nt == 1) tc_commit_elect(&q_empty);   // last read of this item's Q and dO
+      for (int j = 0; j < nt; ++j) {
+        const int t = t0 + j;
+        if (j + 1 < nt) {
+          if (!(ok = issue_s(t + 1) && issue_dp(t + 1))) break;
+          if (j + 2 == nt) tc_commit_elect(&q_empty);
+        }
+        if (!warp_wait(&ds_full[t & 1], (t >> 1) & 1, wc) || (j == 0 && n > 0 && !warp_wait(&dq_free, (n - 1) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t kmn = smem_desc_sw128(sbase + C::K_OFF + (t % kQNSK) * C::TILE, C::CHUNK, 1024);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_elect(tmem + kTQ, tmem + kTS + (t & 1) * 128 + ks * 8, kmn + (uint64_t)(ks * 2048 >> 4), C::ID_Q,
+                       (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit_elect(&k_empty[t % kQNSK]);
+      }
+      if (!ok) break;
+      tc_commit_elect(&dq_ready);
+      t0 += nt;
+    }
+    if (issued) {
+      tc_commit_elect(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0, a.timeout_ns);
+    }
+  } else if (warp >= 2 && warp <= 9) {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3, hw = (warp - 2) >> 2, h = lane >> 4;
+    const int row = quarter * 32 + hw * 16 + (lane & 15);
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32 + hw * 16) << 16);
+    const int g_r = row / R, rr = row % R;
+    const float sl2 = a.sl2;
+    const float log2b = __log2f((float)a.b);
+    constexpr int DH = D / 2;
+    int n = 0, t = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < a.total_items; it += gridDim.x, ++n) {
+      const Item I = decode_item<G>(a, it);
+      const int2 qs = q_span<R>(a, I, g_r);
+      const bool row_valid = rr < qs.y;
+      const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
+      const float2 mine = row_valid ? b.dl[tok] : make_float2(INFINITY, 0.f);
+      const uint32_t* rbits = nullptr;
+      int pb0 = -1, pb1 = -1;
+      float d0 = 0.f, d1 = 0.f;
+      if (I.kind == 2) {
+        const int f = I.slot0 + g_r;
+        if (f < a.n_flat) rbits = a.bits + ((size_t)I.bh * a.n_flat + f) * a.words;
+        if (a.L_src % a.b) {
+          pb0 = a.T_src - 1;
+          d0 = (__log2f((float)(a.L_src % a.b)) - log2b) / sl2;
+        }
+        if ((a.L_ctx % a.b) && a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1) {
+          pb1 = a.T_kv - 1;
+          d1 = (__log2f((float)(a.L_ctx % a.b)) - log2b) / sl2;
+        }
+      }
+      ItemCounts ic;
+      ic.src_tail = a.L_src - (a.T_src - 1) * a.b;
+      ic.kv_tail = a.b;
+      if (a.ctx_sel[(size_t)I.bh * a.K_sel + a.K_sel - 1] == a.T_ctx - 1) ic.kv_tail = a.L_ctx - (a.T_ctx - 1) * a.b;
+      int jm0 = -1, jm1 = -1;
+      if (I.kind == 1) {
+        if (ic.src_tail != a.b) jm0 = (a.T_src - 1) / G;
+        jm1 = (a.T_kv - 1) / G;
+      }
+      int ekk[G];
+      load_exact<G>(a, I, 0, ekk);
+      for (int j = 0; j < I.ntiles; ++j, ++t) {
+        TileMeta cur;
+        if (I.kind == 2 || j == jm0 || j == jm1) {
+          cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
+          load_exact<G>(a, I, j + 1, ekk);
+        } else {
+          cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
+          cur.pooled = 0;
+          cur.masked = 0;
+        }
+        const int buf = t & 1;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sd_full[buf], (t >> 1) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[2][32], dr[2][32];
+        tmem_ld16x2_32<64>(trow + kTS + buf * 128, sr[0]);
+        tmem_ld16x2_32<64>(trow + kTS + buf * 128 + 32, sr[1]);
+        tmem_ld16x2_32<64>(trow + kTP, dr[0]);
+        tmem_ld16x2_32<64>(trow + kTP + 32, dr[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&dp_free);   // dP of the next tile may overwrite the buffer
+        float s[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        if (cur.masked) {
+          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = ((((c < 32) ? w0 : w1) >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+          if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
+            const int kk0 = (j - a.n_exact) * 128 + 64 * h;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
+          }
+        }
+        const float neg = (cur.pooled ? log2b : 0.f) - mine.x;
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = ex2(fmaf(s[c], sl2, neg)), p1 = ex2(fmaf(s[c + 1], sl2, neg));
+          const float g0 = p0 * (__uint_as_float(dr[c >> 5][c & 31]) - mine.y);
+          const float g1 = p1 * (__uint_as_float(dr[(c + 1) >> 5][(c + 1) & 31]) - mine.y);
+          pk[c >> 1] = pack_bf16x2(g0, g1);
+        }
+        tmem_st16x2_32<32>(trow + kTS + buf * 128, pk);   // dS keys 64h..64h+63 -> columns 32h..32h+31
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ds_full[buf]);
+      }
+      if (!ok) break;
+      // epilogue: dQ = s * (dS K summed over the tiles), this thread's DH columns
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&dq_ready, n & 1, wc))) break;
+      tc_fence_after();
+      uint32_t o[DH / 32][32];
+#pragma unroll
+      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld16x2_32<DH>(trow + kTQ + 32 * c0, o[c0]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&dq_free);
+      if (row_valid) {
+        const float sc = b.scale;
+        uint4* dst = reinterpret_cast<uint4*>(b.dq + tok * D + DH * h);
+#pragma unroll
+        for (int c = 0; c < DH; c += 8) {
+          const uint32_t* oc = &o[c >> 5][c & 31];
+          dst[c / 8] = make_uint4(pack_bf16x2(sc * __uint_as_float(oc[0]), sc * __uint_as_float(oc[1])),
+                                  pack_bf16x2(sc * __uint_as_float(oc[2]), sc * __uint_as_float(oc[3])),
+                                  pack_bf16x2(sc * __uint_as_float(oc[4]), sc * __uint_as_float(oc[5])),
+                                  pack_bf16x2(sc * __uint_as_float(oc[6]), sc * __uint_as_float(oc[7])));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <int D, int R>
+static cudaError_t launch_t(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sms, cudaStream_t st) {
+  using KC = KvCfg<D, R>;
+  using QC = QCfg<D, R>;
+  static bool attr_done = false;   // per template instance; set once per process
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_kv_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KC::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QC::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const size_t rows = (size_t)d.BH * d.L;
+  const int pgrid = (int)std::max<size_t>(1, std::min<size_t>((rows * (D / 8) + 255) / 256, (size_t)sms * 16));
+  bwd_prep_kernel<D><<<pgrid, 256, 0, st>>>(reinterpret_cast<const uint4*>(b.o), reinterpret_cast<const uint4*>(b.dout),
+                                            b.lse, b.dl, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (d.K_sel < d.T_ctx) {
+    bwd_zero_unkept_kernel<<<dim3(d.BH, d.T_ctx), 128, 0, st>>>(b.a.ctx_sel, d.K_sel, d.L, d.L_src, d.L_ctx, d.b, D,
+                                                                 reinterpret_cast<uint4*>(b.dk),
+                                                                 reinterpret_cast<uint4*>(b.dv));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (b.has_pooled) {
+    b.kv_pooled = 1;
+    b.kv_tiles = d.T_kv_pad / 128;
+    b.kv_total = d.BH * b.kv_tiles;
+    bwd_kv_kernel<D, R><<<std::min(sms, b.kv_total), kKvThreads, KC::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                                  maps[4], maps[5], b);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  b.kv_pooled = 0;
+  b.kv_tiles = (d.T_kv + KC::G - 1) / KC::G;
+  b.kv_total = d.BH * b.kv_tiles;
+  bwd_kv_kernel<D, R><<<std::min(sms, b.kv_total), kKvThreads, KC::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                                maps[4], maps[5], b);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_q_kernel<D, R><<<std::min(sms, b.a.total_items), kQThreads, QC::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                                   maps[4], maps[5], b);
+  return cudaGetLastError();
+}
+
+}  // namespace bwd
+
+cudaError_t launch_backward(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sm_count, cudaStream_t st) {
+  if (d.D == 128 && d.b == 64) return bwd::launch_t<128, 64>(d, maps, b, sm_count, st);
+  if (d.D == 128 && d.b == 32) return bwd::launch_t<128, 32>(d, maps, b, sm_count, st);
+  if (d.D == 64 && d.b == 64) return bwd::launch_t<64, 64>(d, maps, b, sm_count, st);
+  if (d.D == 64 && d.b == 32) return bwd::launch_t<64, 32>(d, maps, b, sm_count, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace isa

@@ -54,15 +54,35 @@ struct AttnArgs {
   int inject;
 };
 
+// Argument block of the backward kernels (isa_bwd.cu).  `a` carries the
+// plan, the sizes and the forward's sparse work list (mode 0).
+struct BwdArgs {
+  AttnArgs a;
+  const __nv_bfloat16* o;      // forward output [BH*L, D]
+  const __nv_bfloat16* dout;   // gradient of the output [BH*L, D]
+  const float* lse;            // forward natural-log normalisers [BH*L]
+  float2* dl;                  // per query row: (lse * log2 e, rowsum(dout * o))
+  float* dKc;                  // [BH, T_kv_pad, D] gradient of the pooled keys (scaled)
+  float* dVc;                  // [BH, T_kv_pad, D] gradient of the pooled values
+  __nv_bfloat16 *dq, *dk, *dv; // [BH*L, D]
+  float scale;                 // softmax scale s
+  int has_pooled;              // some flat block has pooled columns (dKc/dVc are filled)
+  int kv_pooled;               // key/value-stationary launch over pooled rows (1) or kept blocks (0)
+  int kv_tiles;                // key/value tiles per head of that launch
+  int kv_total;                // BH * kv_tiles
+};
+
 // launchers (host)
 cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
                         cudaStream_t st);
 cudaError_t prepare_plan_kernels();
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
+cudaError_t launch_backward(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sm_count, cudaStream_t st);
 size_t rope_table_bytes(const Dims& d);
 cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
                         int sm_count, cudaStream_t st);
 void set_last_error(const char* msg);
+isa_status bind_device_of(const void* ptr, const char* name);
 
 constexpr int kMaxT = 8192;      // blocks per head
 constexpr int kMaxTkv = 6144;    // kept blocks per head

@@ -47,6 +47,11 @@ extern "C" isa_status isa_forward_static(const isa_params* p, const void* q, con
     isa::set_last_error(msg);
     return ISA_ERR_WORKSPACE;
   }
+  if (!q) {
+    isa::set_last_error("q is NULL");
+    return ISA_ERR_INVALID_ARG;
+  }
+  if ((s = isa::bind_device_of(q, "q")) != ISA_OK) return s;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {

@@ -159,6 +159,40 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
 isa_status isa_forward_static(const isa_params* p, const void* q, const void* k, const void* v, void* out,
                               float* lse, void* stream);
 
+/* Workspace of isa_backward: (lse * log2 e, rowsum(dout * out)) per query
+ * row (8 bytes each) and fp32 gradients of the pooled keys and values
+ * (2 * B*H * T_kv_pad * D * 4 bytes), each 256-byte aligned. */
+isa_status isa_backward_workspace_size(const isa_params* p, size_t* bytes);
+
+/* Gradients of the isa_forward output with respect to Q, K and V, for the
+ * loss sum(dout * out), with the plan in `ws` held fixed.  The summary card
+ * ("Core method", innovation (c)) and the techwalker.com article (training
+ * section) state that ISA has a forward and a backward implementation and is
+ * trained end to end; they print no gradient formulas.  These are the
+ * gradients of the forward as computed: the plan's choices (kept context
+ * blocks, sharp/flat split, exact lists) carry no gradient, a flat block's
+ * pooled key Kc_j / value Vc_j (the mean of block j's n_j tokens) passes its
+ * gradient to each token of block j divided by n_j, and the count weight n_j
+ * is a constant.  With P the softmax weights of a query row over its columns,
+ * dP = dout V^T and Delta = rowsum(dout * out):
+ *   dS = P (dP - Delta),  dq = s dS K,  dk = s dS^T Q,  dv = P^T dout.
+ *   q, k, v, ws : the inputs and the plan of the forward call
+ *   out         : device bf16 [B,H,L,D], the forward's output
+ *   lse         : device fp32 [B,H,L], the forward's lse (isa_forward with lse != NULL)
+ *   dout        : device bf16 [B,H,L,D]
+ *   dq, dk, dv  : device bf16 [B,H,L,D]; every element is written (tokens of
+ *                 context blocks that were not kept get dk = dv = 0)
+ *   bws         : device, >= isa_backward_workspace_size bytes, 256-byte
+ *                 aligned; caller-owned scratch, rewritten by every call
+ * P is recomputed from lse (no attention matrix is stored); products run in
+ * bf16 on the tensor cores with fp32 accumulation, P and dS rounded to bf16.
+ * Launches 5 kernels (4 when every kept block is exact for every flat
+ * block, or no block is flat; one more when every context block is kept).
+ * Device timeouts go to the plan's status word, as for isa_forward. */
+isa_status isa_backward(const isa_params* p, const void* q, const void* k, const void* v, const void* ws,
+                        size_t ws_bytes, const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                        void* dv, void* bws, size_t bws_bytes, void* stream);
+
 /* Workspace of isa_rope: the cos/sin table, max(L_src, L_ctx) * D/2 float
  * pairs (8 bytes each). */
 isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes);

@@ -153,3 +153,31 @@ def test_product_path_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "isa_oracle" not in text, f
+
+
+def test_backward_arguments_rejected_before_launch(isa):
+    """isa_backward checks every pointer, the plan workspace and its own
+    workspace on the host (fake device addresses: nothing may be launched)."""
+    lib = isa.load_library()
+    p = isa.make_params(1, 2, 64, 300, 100)
+    n = isa.workspace_size(p)
+    nb = isa.backward_workspace_size(p)
+    BH, L, T_kv_pad = 2, 400, 128
+    # (lse*log2e, Delta) per row, then dKc and dVc in fp32, each 256-byte aligned
+    a256 = lambda x: (x + 255) // 256 * 256
+    assert nb == a256(BH * L * 8) + 2 * a256(BH * T_kv_pad * 64 * 4)
+    a = 1 << 20
+    args = [ctypes.byref(p), a, a, a, a, n, a, a, a, a, a, a, a, nb, None]
+
+    def call(**kw):
+        x = list(args)
+        for i, val in kw.items():
+            x[int(i[1:])] = val
+        return lib.isa_backward(*x)
+
+    assert call(_8=None) == 1 and b"dout is NULL" in lib.isa_last_error()
+    assert call(_10=a + 8) == 1 and b"dk" in lib.isa_last_error()
+    assert call(_7=a + 2) == 1 and b"lse" in lib.isa_last_error()
+    assert call(_12=a + 16) == 1 and b"backward workspace" in lib.isa_last_error()
+    assert call(_13=nb - 1) == 3
+    assert call(_5=n - 1) == 3

@@ -21,7 +21,8 @@ float64 values the oracle works on.
 
 Random streams: each (tensor, batch*H + head) pair draws from its own
 ``numpy.random.PCG64`` seeded with the entropy list ``[seed, stream, bh]``,
-stream 0/1/2 = Q/K/V, 3 = per-cluster noise level, 4 = per-head Q temperature.
+stream 0/1/2 = Q/K/V, 3 = per-cluster noise level, 4 = per-head Q temperature,
+5 = the upstream gradient dout of the backward (standard normal per element).
 A head can therefore be regenerated on its own, which is how the tests fetch
 oracle inputs for sampled heads of the large workloads.
 """
@@ -195,6 +196,23 @@ def generate_bits(w: Workload, heads: Optional[List[int]] = None,
     return q, k, v
 
 
+def dout_head_bits(w: Workload, bh: int) -> np.ndarray:
+    """bf16 bits of the upstream gradient dout [L, D] of head bh: independent
+    standard normal values (the loss is sum(dout * out))."""
+    g = _rng(w.seed, 5, bh)
+    return f32_to_bf16_bits(g.standard_normal((w.L, w.D), dtype=np.float32))
+
+
+def generate_dout_bits(w: Workload, heads: Optional[List[int]] = None) -> np.ndarray:
+    """dout bits, [B, H, L, D] (heads=None) or [len(heads), L, D]."""
+    hs = list(range(w.BH)) if heads is None else list(heads)
+    out = np.empty((len(hs), w.L, w.D), np.uint16)
+    with _cf.ThreadPoolExecutor(max_workers=min(len(hs), os.cpu_count() or 1) or 1) as ex:
+        for i, x in zip(range(len(hs)), ex.map(lambda h: dout_head_bits(w, h), hs)):
+            out[i] = x
+    return out.reshape(w.B, w.H, w.L, w.D) if heads is None else out
+
+
 def sample_blocks(w: Workload, n_heads: int, n_blocks: int, seed: int = 7) -> List[Tuple[int, int]]:
     """Seeded sample of (bh, query-block) pairs for spot checks at full size."""
     T = -(-w.L_src // w.block) + -(-w.L_ctx // w.block)
@@ -218,6 +236,7 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "Workload", "named_workloads", "f32_to_bf16_bits", "bf16_to_f32", "bf16_to_f64",
-    "head_f32", "head_bits", "generate_bits", "sample_blocks", "flops_dense", "ceil_div",
+    "head_f32", "head_bits", "generate_bits", "dout_head_bits", "generate_dout_bits", "sample_blocks",
+    "flops_dense", "ceil_div",
     "CLUSTER",
 ]
