@@ -343,7 +343,8 @@ static isa_status run_attention(const Dims& d, int mode, const void* q, const vo
   return ISA_OK;
 }
 
-// Byte offsets of the backward workspace: per query row (lse2, Delta), then
+// Byte offsets of the backward workspace: (lse2, Delta) per row of every
+// query block ([BH, T, b], padded past each block's end), then
 // the fp32 gradients of the pooled keys and values.
 struct BwdLayout {
   size_t dl, dKc, dVc, total;
@@ -352,7 +353,7 @@ struct BwdLayout {
 static BwdLayout bwd_layout(const Dims& d) {
   BwdLayout L{};
   L.dl = 0;
-  L.dKc = align256((size_t)d.BH * d.L * 8);
+  L.dKc = align256((size_t)d.BH * d.T * d.b * 8);
   L.dVc = L.dKc + align256((size_t)d.BH * d.T_kv_pad * d.D * 4);
   L.total = L.dVc + align256((size_t)d.BH * d.T_kv_pad * d.D * 4);
   return L;

@@ -52,24 +52,36 @@ __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
   return acc;
 }
 
-// dl[r] = (lse[r] * log2 e, sum_d dout[r, d] * o[r, d]); D/8 lanes per row,
-// grid-stride over the rows (the loop bound is warp-uniform).
+// dl[(bh*T + j)*b + r] = (lse * log2 e, sum_d dout * o) of row r of block j
+// of head bh, and (inf, 0) for r past the block's end, so that every query
+// block's entries are one aligned run of b float2.  D/8 lanes per entry,
+// grid-stride over the BH*T*b entries (the loop bound is warp-uniform).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                                                        const float* __restrict__ lse, float2* __restrict__ dl,
-                                                       size_t rows) {
+                                                       int T, int b, int L, int L_src, int L_ctx, int T_src,
+                                                       size_t entries) {
   constexpr int LPR = D / 8;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
   const size_t warp = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const size_t nwarps = ((size_t)gridDim.x * blockDim.x) >> 5;
-  for (size_t r0 = warp * RPW; r0 < rows; r0 += nwarps * RPW) {
-    const size_t r = r0 + lane / LPR;
+  for (size_t e0 = warp * RPW; e0 < entries; e0 += nwarps * RPW) {
+    const size_t e = e0 + lane / LPR;
+    bool valid = false;
+    size_t row = 0;
+    if (e < entries) {
+      const size_t bh = e / ((size_t)T * b);
+      const int j = (int)((e / b) % T), r = (int)(e % b);
+      const int2 sp = block_span(j, L_src, L_ctx, b, T_src);
+      valid = r < sp.y;
+      row = bh * L + sp.x + r;
+    }
     float acc = 0.f;
-    if (r < rows) acc = dot_bf16x8(o[r * LPR + lane % LPR], dout[r * LPR + lane % LPR]);
+    if (valid) acc = dot_bf16x8(o[row * LPR + lane % LPR], dout[row * LPR + lane % LPR]);
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-    if (r < rows && lane % LPR == 0) dl[r] = make_float2(lse[r] * kLog2e, acc);
+    if (e < entries && lane % LPR == 0) dl[e] = valid ? make_float2(lse[row] * kLog2e, acc) : make_float2(INFINITY, 0.f);
   }
 }
 
@@ -114,14 +126,21 @@ __global__ void __launch_bounds__(128) bwd_zero_unkept_kernel(const int* __restr
 //   S^T = K Q^T, dP^T = V dO^T         (SS, M=128, N=64, K=D)
 //   P^T = 2^(S^T s log2e + w_j - lse2), dS^T = P^T (dP^T - Delta)   (softmax warps)
 //   dV += P^T dO, dK += dS^T Q         (TS: P^T / dS^T read as bf16 from TMEM)
-// Roles (320 threads, one CTA per SM): warp 0 lane 0 TMA producer (the tile,
+// Roles (576 threads, one CTA per SM): warp 0 lane 0 TMA producer (the tile,
 // the query/dO steps and their metadata), warp 1 MMA issuer (converged, one
-// elected lane), warps 2..9: warp w owns TMEM lanes 32*(w%4).. and query
-// columns 32*((w-2)/4).. of each step, and writes the epilogue.
-constexpr int kKvThreads = 320;
+// elected lane), warps 2..17: warp w owns TMEM lanes 32*(w%4).. and query
+// columns 16*((w-2)/4).. of each step (four warps per lane quarter, so that
+// each scheduler interleaves four of them), and writes the epilogue.
+constexpr int kKvSoft = 16;                      // softmax warps
+constexpr int kKvThreads = 64 + 32 * kKvSoft;
 constexpr int kNSQ = 3;           // query/dO step stages
-constexpr uint32_t kTST = 0;      // S^T then P^T (bf16): two buffers of 64 columns
-constexpr uint32_t kTDP = 128;    // dP^T then dS^T (bf16): two buffers of 64 columns
+// TMEM: S^T and dP^T of two steps (step u in buffer u % 2, so the next
+// step's products run while the softmax warps work on this one); each
+// softmax warp packs its bf16 P^T / dS^T into the first half of the 16
+// fp32 columns it has just read, where the dV / dK products take them as
+// the A operand; then dV and dK.
+constexpr uint32_t kTST = 0;      // S^T then P^T, two buffers of 64 columns
+constexpr uint32_t kTDP = 128;    // dP^T then dS^T, two buffers of 64 columns    // two buffers of 64 columns: P^T (bf16 pairs) at +0, dS^T at +32
 constexpr uint32_t kTDV = 256;    // dV accumulator (D columns); dK at kTDV + D
 
 template <int D, int R>
@@ -138,7 +157,9 @@ struct KvCfg {
   static constexpr uint32_t V_OFF = TILE;
   static constexpr uint32_t Q_OFF = 2 * TILE;
   static constexpr uint32_t DO_OFF = Q_OFF + kNSQ * QTILE;
-  static constexpr uint32_t SMEM_USED = DO_OFF + kNSQ * QTILE + 1024;
+  static constexpr uint32_t DL_OFF = DO_OFF + kNSQ * QTILE;   // (lse2, Delta) of the 64 step rows
+  static constexpr uint32_t DL_STAGE = 64 * 8;
+  static constexpr uint32_t SMEM_USED = DL_OFF + kNSQ * DL_STAGE + 1024;
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits on an SM
   static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t ID_T = idesc_bf16_f32(128, 64, 0);
@@ -146,6 +167,7 @@ struct KvCfg {
 };
 
 struct StepMeta {
+  int blk[2];             // block ids of the step's query blocks
   int start[2], cnt[2];   // token start and valid rows of the step's query blocks
   uint32_t m[2][4];       // tile rows each query block attends (bit r of m[g][r/32])
   int last;               // last step of the item
@@ -154,6 +176,7 @@ struct StepMeta {
 __device__ __forceinline__ void clear_meta(StepMeta& m) {
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
+    m.blk[g] = 0;
     m.start[g] = 0;
     m.cnt[g] = 0;
 #pragma unroll
@@ -190,12 +213,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sd_full[i], 1);
-      mbar_init(&ds_full[i], 256);
-    }
+    mbar_init(&sd_full[0], 1);
+    mbar_init(&sd_full[1], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&ds_full[i], 32 * kKvSoft);
     mbar_init(&acc_ready, 1);
-    mbar_init(&acc_free, 256);
+    mbar_init(&acc_free, 32 * kKvSoft);
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -214,80 +236,112 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const WaitCtl wc{&abort_flag, a.status, a.timeout_ns};
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- producer
-      int kv_cnt = 0, qcnt[kNSQ];
-      for (int i = 0; i < kNSQ; ++i) qcnt[i] = 0;
-      int u = 0, n = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
-        const int bh = it / b.kv_tiles, tile = it % b.kv_tiles;
-        if (n >= 1 && !mbar_wait(&kv_empty, (n - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&kv_full, 2 * C::TILE);
-        ++kv_cnt;
-        for (int g = 0; g < G; ++g) {
-          int row;
-          if (pooled) {
-            row = bh * a.T_kv_pad + tile * 128 + g * R;
-          } else {
-            const int kk = tile * G + g;
-            row = bh * a.L;
-            if (kk < a.T_kv) row += block_span(a.kept[(size_t)bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src).x;
-          }
-          for (int c = 0; c < C::NCH; ++c) {
-            tma_load_2d(sgen + C::K_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_kp : &tm_k, c * 64, row, &kv_full);
-            tma_load_2d(sgen + C::V_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_vp : &tm_v, c * 64, row, &kv_full);
-          }
-        }
-        // Steps are published one behind, so that the last one can be marked.
-        StepMeta pend, grp;
-        bool have = false;
-        int ng = 0;
-        auto emit = [&](const StepMeta& m, int last) -> bool {
-          const int s = u % kNSQ;
-          if (u >= kNSQ && !mbar_wait(&q_empty[s], ((u / kNSQ) - 1) & 1, wc)) return false;
-          meta[s] = m;
-          meta[s].last = last;   // published by the arrive below (release), read after q_full (acquire)
-          mbar_arrive_expect_tx(&q_full[s], 2 * C::QTILE);
-          ++qcnt[s];
-          for (int g = 0; g < GQ; ++g) {
-            const int row = bh * a.L + (m.cnt[g] > 0 ? m.start[g] : 0);
+    // ------------------------------------------------------------ producer
+    // The whole warp finds the steps (32 sharp ids or 32 flat blocks' exact
+    // bitmaps per round of loads, matches picked by ballot); lane 0 publishes
+    // them and issues every copy.
+    int kv_cnt = 0, qcnt[kNSQ];
+    for (int i = 0; i < kNSQ; ++i) qcnt[i] = 0;
+    int u = 0, n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
+      const int bh = it / b.kv_tiles, tile = it % b.kv_tiles;
+      if (lane == 0) {
+        if (n >= 1 && !mbar_wait(&kv_empty, (n - 1) & 1, wc)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(&kv_full, 2 * C::TILE);
+          ++kv_cnt;
+          for (int g = 0; g < G; ++g) {
+            int row;
+            if (pooled) {
+              row = bh * a.T_kv_pad + tile * 128 + g * R;
+            } else {
+              const int kk = tile * G + g;
+              row = bh * a.L;
+              if (kk < a.T_kv) row += block_span(a.kept[(size_t)bh * a.T_kv + kk], a.L_src, a.L_ctx, a.b, a.T_src).x;
+            }
             for (int c = 0; c < C::NCH; ++c) {
-              tma_load_2d(sgen + C::Q_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_q, c * 64, row,
-                          &q_full[s]);
-              tma_load_2d(sgen + C::DO_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_do, c * 64, row,
-                          &q_full[s]);
+              tma_load_2d(sgen + C::K_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_kp : &tm_k, c * 64, row, &kv_full);
+              tma_load_2d(sgen + C::V_OFF + c * C::CHUNK + g * C::BOX, pooled ? &tm_vp : &tm_v, c * 64, row, &kv_full);
             }
-          }
-          ++u;
-          return true;
-        };
-        auto push = [&](const StepMeta& m) -> bool {
-          const bool r = have ? emit(pend, 0) : true;
-          pend = m;
-          have = true;
-          return r;
-        };
-        if (!pooled) {
-          // sharp blocks attend every kept block: all rows of the tile
-          for (int s0 = 0; ok && s0 < a.n_sharp; s0 += GQ) {
-            StepMeta m;
-            clear_meta(m);
-            for (int g = 0; g < GQ; ++g) {
-              if (s0 + g >= a.n_sharp) break;
-              const int2 sp = block_span(a.sharp[(size_t)bh * a.n_sharp + s0 + g], a.L_src, a.L_ctx, a.b, a.T_src);
-              m.start[g] = sp.x;
-              m.cnt[g] = sp.y;
-              for (int w = 0; w < 4; ++w) m.m[g][w] = 0xFFFFFFFFu;
-            }
-            ok = push(m);
           }
         }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      // Steps are published one behind, so that the last one can be marked
+      // (lane 0's copies of pend/grp are the live ones).
+      StepMeta pend, grp;
+      bool have = false;
+      int ng = 0;
+      clear_meta(grp);
+      auto emit = [&](const StepMeta& m, int last) -> bool {
+        const int s = u % kNSQ;
+        if (u >= kNSQ && !mbar_wait(&q_empty[s], ((u / kNSQ) - 1) & 1, wc)) return false;
+        meta[s] = m;
+        meta[s].last = last;   // published by the arrive below (release), read after q_full (acquire)
+        mbar_arrive_expect_tx(&q_full[s], 2 * C::QTILE + C::DL_STAGE);
+        ++qcnt[s];
+        for (int g = 0; g < GQ; ++g) {
+          const int row = bh * a.L + (m.cnt[g] > 0 ? m.start[g] : 0);
+          bulk_load_1d(sgen + C::DL_OFF + s * C::DL_STAGE + g * R * 8,
+                       b.dl + ((size_t)bh * (a.T_src + a.T_ctx) + m.blk[g]) * R, R * 8, &q_full[s]);
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_2d(sgen + C::Q_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[s]);
+            tma_load_2d(sgen + C::DO_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_do, c * 64, row,
+                        &q_full[s]);
+          }
+        }
+        ++u;
+        return true;
+      };
+      auto push = [&](const StepMeta& m) -> bool {
+        const bool r = have ? emit(pend, 0) : true;
+        pend = m;
+        have = true;
+        return r;
+      };
+      // query block blk (row mask mw) joins the step being assembled; lane 0 only
+      auto add = [&](int blk, const uint32_t (&mw)[4]) -> bool {
+        const int2 sp = block_span(blk, a.L_src, a.L_ctx, a.b, a.T_src);
+        grp.blk[ng] = blk;
+        grp.start[ng] = sp.x;
+        grp.cnt[ng] = sp.y;
+        for (int w = 0; w < 4; ++w) grp.m[ng][w] = mw[w];
+        if (++ng < GQ) return true;
+        const bool r = push(grp);
         clear_meta(grp);
-        for (int f = 0; ok && f < a.n_flat; ++f) {
+        ng = 0;
+        return r;
+      };
+      if (!pooled) {
+        // sharp blocks attend every kept block: all rows of the tile
+        const uint32_t all[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+        for (int base = 0; ok && base < a.n_sharp; base += 32) {
+          const int idx = base + lane;
+          const int blk = idx < a.n_sharp ? a.sharp[(size_t)bh * a.n_sharp + idx] : 0;
+          const int cnt = min(32, a.n_sharp - base);
+          for (int j = 0; j < cnt; ++j) {
+            const int bj = __shfl_sync(0xFFFFFFFFu, blk, j);
+            if (lane == 0) ok = add(bj, all);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+          }
+        }
+        if (lane == 0 && ok && ng > 0) {   // the sharp blocks' last partial step
+          ok = push(grp);
+          clear_meta(grp);
+          ng = 0;
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      }
+      for (int base = 0; ok && base < a.n_flat; base += 32) {
+        const int f = base + lane;
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        int blk = 0;
+        if (f < a.n_flat) {
           const uint32_t* fb = a.bits + ((size_t)bh * a.n_flat + f) * a.words;
-          uint32_t mw[4];
-          bool any = false;
           if (pooled) {
             // pooled rows tile*128 + r, minus the flat block's exact blocks
             for (int w = 0; w < 4; ++w) {
@@ -295,34 +349,39 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               const int rem = a.T_kv - (tile * 128 + 32 * w);
               const uint32_t range = rem >= 32 ? 0xFFFFFFFFu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
               mw[w] = range & ~(wi < a.words ? fb[wi] : 0u);
-              any = any || mw[w] != 0u;
             }
           } else {
             // exact blocks among kept positions tile*G .. tile*G+G-1 (one word)
             const int k0 = tile * G;
             const uint32_t gm = (fb[k0 >> 5] >> (k0 & 31)) & ((1u << G) - 1u);
-            any = gm != 0u;
             for (int w = 0; w < 4; ++w) mw[w] = ((gm >> ((32 * w) / R)) & 1u) ? 0xFFFFFFFFu : 0u;
           }
-          if (!any) continue;
-          const int2 sp = block_span(a.flat[(size_t)bh * a.n_flat + f], a.L_src, a.L_ctx, a.b, a.T_src);
-          grp.start[ng] = sp.x;
-          grp.cnt[ng] = sp.y;
-          for (int w = 0; w < 4; ++w) grp.m[ng][w] = mw[w];
-          if (++ng == GQ) {
-            ok = push(grp);
-            clear_meta(grp);
-            ng = 0;
-          }
+          if (mw[0] | mw[1] | mw[2] | mw[3]) blk = a.flat[(size_t)bh * a.n_flat + f];
         }
-        if (ok && ng > 0) ok = push(grp);
+        uint32_t bal = __ballot_sync(0xFFFFFFFFu, (mw[0] | mw[1] | mw[2] | mw[3]) != 0u);
+        while (bal) {
+          const int src = __ffs(bal) - 1;
+          bal &= bal - 1;
+          uint32_t m4[4];
+          for (int w = 0; w < 4; ++w) m4[w] = __shfl_sync(0xFFFFFFFFu, mw[w], src);
+          const int bj = __shfl_sync(0xFFFFFFFFu, blk, src);
+          if (lane == 0) ok = add(bj, m4);
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          if (!ok) break;
+        }
+      }
+      if (lane == 0 && ok) {
+        if (ng > 0) ok = push(grp);
         if (ok && !have) {
           clear_meta(pend);   // no query attends the tile: one empty step writes zeros
           have = true;
         }
         if (ok) ok = emit(pend, 1);
       }
-      // let every copy in flight land before the CTA can exit
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    }
+    // let every copy in flight land before the CTA can exit
+    if (lane == 0) {
       if (kv_cnt) mbar_wait_drain(&kv_full, (kv_cnt - 1) & 1, a.timeout_ns);
       for (int i = 0; i < kNSQ; ++i)
         if (qcnt[i]) mbar_wait_drain(&q_full[i], (qcnt[i] - 1) & 1, a.timeout_ns);
@@ -336,22 +395,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // S^T and dP^T of step uu into buffer uu % 2
     auto issue_t = [&](int uu) -> bool {
       const int s = uu % kNSQ;
-      if (!warp_wait(&q_full[s], (uu / kNSQ) & 1, wc)) return false;
+      if (!warp_wait(&q_full[s], (uu / kNSQ) & 1, wc))
+        return false;
       tc_fence_after();
       const uint64_t qd = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, 16, 1024);
       const uint64_t dd = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, 16, 1024);
-      const uint32_t col = (uu & 1) * 64;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
         const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
-        mma_ss_elect(tmem + kTST + col, kdesc + oa, qd + ob, C::ID_T, ks > 0);
+        mma_ss_elect(tmem + kTST + (uu & 1) * 64, kdesc + oa, qd + ob, C::ID_T, ks > 0);
       }
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
         const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
-        mma_ss_elect(tmem + kTDP + col, vdesc + oa, dd + ob, C::ID_T, ks > 0);
+        mma_ss_elect(tmem + kTDP + (uu & 1) * 64, vdesc + oa, dd + ob, C::ID_T, ks > 0);
       }
       issued = true;
       tc_commit_elect(&sd_full[uu & 1]);
@@ -375,17 +434,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc_fence_after();
         const uint64_t qmn = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, C::QCHUNK, 1024);
         const uint64_t dmn = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, C::QCHUNK, 1024);
-        const uint32_t col = (u & 1) * 64;
-        // packed bf16 P^T / dS^T: warp half h holds query columns 32h..32h+31
-        // in its buffer's columns 32h..32h+15
+        const uint32_t pk = (u & 1) * 64;
+        // packed bf16 P^T / dS^T: query columns 16q..16q+15 (one K step) sit
+        // in the buffer's columns 16q..16q+7
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts_elect(tmem + kTDV, tmem + kTST + col + (ks >> 1) * 32 + (ks & 1) * 8,
-                       dmn + (uint64_t)(ks * 2048 >> 4), C::ID_A, (!first || ks > 0) ? 1u : 0u);
+          mma_ts_elect(tmem + kTDV, tmem + kTST + pk + ks * 16, dmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
+                       (!first || ks > 0) ? 1u : 0u);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts_elect(tmem + kTDV + D, tmem + kTDP + col + (ks >> 1) * 32 + (ks & 1) * 8,
-                       qmn + (uint64_t)(ks * 2048 >> 4), C::ID_A, (!first || ks > 0) ? 1u : 0u);
+          mma_ts_elect(tmem + kTDV + D, tmem + kTDP + pk + ks * 16, qmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
+                       (!first || ks > 0) ? 1u : 0u);
         tc_commit_elect(&q_empty[s]);
         ++u;
         if (last) break;
@@ -400,13 +459,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int quarter = warp & 3, hw = (warp - 2) >> 2;
+    const int quarter = warp & 3, qd = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                      // tile row = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int gq = (R == 32) ? hw : 0;                      // this thread's query block of a step
-    const int coff = (R == 32) ? 0 : 32 * hw;               // its first column within that block
+    const int gq = (R == 32) ? (qd >> 1) : 0;               // this thread's query block of a step
+    const int coff = (R == 32) ? 16 * (qd & 1) : 16 * qd;   // its first column within that block
     const float sl2 = a.sl2;
-    constexpr int DH = D / 2;
+    constexpr int DQ = D / 4;                               // epilogue columns of dV and of dK
     int u = 0, n = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
@@ -430,38 +489,42 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           tok = sp.x + r % R;
         }
       }
-      const float2* dlh = b.dl + (size_t)bh * a.L;
       for (;;) {
         const int s = u % kNSQ, buf = u & 1;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sd_full[buf], (u >> 1) & 1, wc))) {
+        // sd_full follows q_full of the same step (the MMAs waited for it);
+        // the q_full test makes the bulk-copied (lse2, Delta) visible here
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sd_full[buf], (u >> 1) & 1, wc) &&
+                                         mbar_wait(&q_full[s], (u / kNSQ) & 1, wc))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int st0 = meta[s].start[gq], cn = meta[s].cnt[gq], last = meta[s].last;
+        const int last = meta[s].last;
         const bool on = row_valid && ((meta[s].m[gq][r >> 5] >> (r & 31)) & 1u);
-        // lane c fetches (lse2, Delta) of column coff + c; shared by shuffles
-        const int c = coff + lane;
-        const float2 mine = c < cn ? dlh[st0 + c] : make_float2(INFINITY, 0.f);
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tl + kTST + buf * 64 + 32 * hw, sv);
-        tmem_ld32(tl + kTDP + buf * 64 + 32 * hw, dp);
-        tmem_wait_ld();
-        uint32_t pp[16], pd[16];
+        uint32_t sv[16], dp[16];
+        tmem_ld16(tl + kTST + buf * 64 + 16 * qd, sv);
+        tmem_ld16(tl + kTDP + buf * 64 + 16 * qd, dp);
+        // (lse2, Delta) of this thread's 16 columns, two columns per 16-byte
+        // broadcast load; rows past a block's end hold (inf, 0), so P = 0 there
+        const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE) + (gq * R + coff) / 2;
+        float4 ld[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float l0 = __shfl_sync(0xFFFFFFFFu, mine.x, e), l1 = __shfl_sync(0xFFFFFFFFu, mine.x, e + 1);
-          const float d0 = __shfl_sync(0xFFFFFFFFu, mine.y, e), d1 = __shfl_sync(0xFFFFFFFFu, mine.y, e + 1);
-          float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, bias - l0));
-          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, bias - l1));
+        for (int e = 0; e < 8; ++e) ld[e] = dls[e];
+        tmem_wait_ld();
+        uint32_t pp[8], pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float4 x = ld[e >> 1];
+          float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, bias - x.x));
+          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, bias - x.z));
           if (!on) p0 = p1 = 0.f;
-          const float g0 = p0 * (__uint_as_float(dp[e]) - d0);
-          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - d1);
+          const float g0 = p0 * (__uint_as_float(dp[e]) - x.y);
+          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - x.w);
           pp[e >> 1] = pack_bf16x2(p0, p1);
           pd[e >> 1] = pack_bf16x2(g0, g1);
         }
-        tmem_st16(tl + kTST + buf * 64 + 32 * hw, pp);
-        tmem_st16(tl + kTDP + buf * 64 + 32 * hw, pd);
+        tmem_st8(tl + kTST + buf * 64 + 16 * qd, pp);
+        tmem_st8(tl + kTDP + buf * 64 + 16 * qd, pd);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ds_full[buf]);
@@ -469,14 +532,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (last) break;
       }
       if (!ok) break;
-      // epilogue: this thread's DH columns of dV and dK for tile row r
+      // epilogue: this thread's DQ columns of dV and dK for tile row r
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_ready, n & 1, wc))) break;
       tc_fence_after();
-      uint32_t gv[DH / 32][32], gk[DH / 32][32];
+      uint32_t gv[DQ / 16][16], gk[DQ / 16][16];
 #pragma unroll
-      for (int c0 = 0; c0 < DH / 32; ++c0) {
-        tmem_ld32(tl + kTDV + hw * DH + 32 * c0, gv[c0]);
-        tmem_ld32(tl + kTDV + D + hw * DH + 32 * c0, gk[c0]);
+      for (int c0 = 0; c0 < DQ / 16; ++c0) {
+        tmem_ld16(tl + kTDV + qd * DQ + 16 * c0, gv[c0]);
+        tmem_ld16(tl + kTDV + D + qd * DQ + 16 * c0, gk[c0]);
       }
       tmem_wait_ld();
       tc_fence_before();
@@ -484,12 +547,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (!row_valid) continue;
       const float sc = b.scale;
       if (pooled) {
-        float4* kd = reinterpret_cast<float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
-        float4* vd = reinterpret_cast<float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
+        float4* kd = reinterpret_cast<float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
+        float4* vd = reinterpret_cast<float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
 #pragma unroll
-        for (int e = 0; e < DH; e += 4) {
-          const uint32_t* k4 = &gk[e >> 5][e & 31];
-          const uint32_t* v4 = &gv[e >> 5][e & 31];
+        for (int e = 0; e < DQ; e += 4) {
+          const uint32_t* k4 = &gk[e >> 4][e & 15];
+          const uint32_t* v4 = &gv[e >> 4][e & 15];
           kd[e >> 2] = make_float4(sc * __uint_as_float(k4[0]), sc * __uint_as_float(k4[1]),
                                    sc * __uint_as_float(k4[2]), sc * __uint_as_float(k4[3]));
           vd[e >> 2] = make_float4(__uint_as_float(v4[0]), __uint_as_float(v4[1]), __uint_as_float(v4[2]),
@@ -498,17 +561,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       } else {
         // this block's share of its pooled-mean gradient: dKc_j / n_j, dVc_j / n_j
         const float inv = 1.f / (float)nj;
-        const float4* kc = reinterpret_cast<const float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
-        const float4* vc = reinterpret_cast<const float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + hw * DH);
-        uint4* kd = reinterpret_cast<uint4*>(b.dk + ((size_t)bh * a.L + tok) * D + hw * DH);
-        uint4* vd = reinterpret_cast<uint4*>(b.dv + ((size_t)bh * a.L + tok) * D + hw * DH);
+        const float4* kc = reinterpret_cast<const float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
+        const float4* vc = reinterpret_cast<const float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
+        uint4* kd = reinterpret_cast<uint4*>(b.dk + ((size_t)bh * a.L + tok) * D + qd * DQ);
+        uint4* vd = reinterpret_cast<uint4*>(b.dv + ((size_t)bh * a.L + tok) * D + qd * DQ);
 #pragma unroll
-        for (int e = 0; e < DH; e += 8) {
+        for (int e = 0; e < DQ; e += 8) {
           float xk[8], xv[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            xk[i] = sc * __uint_as_float(gk[(e + i) >> 5][(e + i) & 31]);
-            xv[i] = __uint_as_float(gv[(e + i) >> 5][(e + i) & 31]);
+            xk[i] = sc * __uint_as_float(gk[(e + i) >> 4][(e + i) & 15]);
+            xv[i] = __uint_as_float(gv[(e + i) >> 4][(e + i) & 15]);
           }
           if (b.has_pooled) {
             const float4 k0 = kc[e >> 2], k1 = kc[(e >> 2) + 1], v0 = vc[e >> 2], v1 = vc[(e >> 2) + 1];
@@ -768,7 +831,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int2 qs = q_span<R>(a, I, g_r);
       const bool row_valid = rr < qs.y;
       const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
-      const float2 mine = row_valid ? b.dl[tok] : make_float2(INFINITY, 0.f);
+      const int qblk = qs.x < a.L_src ? qs.x / a.b : a.T_src + (qs.x - a.L_src) / a.b;
+      const float2 mine = row_valid ? b.dl[((size_t)I.bh * (a.T_src + a.T_ctx) + qblk) * a.b + rr]
+                                    : make_float2(INFINITY, 0.f);
       const uint32_t* rbits = nullptr;
       int pb0 = -1, pb1 = -1;
       float d0 = 0.f, d1 = 0.f;
@@ -895,10 +960,10 @@ static cudaError_t launch_t(const Dims& d, const CUtensorMap* maps, BwdArgs& b, 
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const size_t rows = (size_t)d.BH * d.L;
-  const int pgrid = (int)std::max<size_t>(1, std::min<size_t>((rows * (D / 8) + 255) / 256, (size_t)sms * 16));
+  const size_t entries = (size_t)d.BH * d.T * d.b;
+  const int pgrid = (int)std::max<size_t>(1, std::min<size_t>((entries * (D / 8) + 255) / 256, (size_t)sms * 16));
   bwd_prep_kernel<D><<<pgrid, 256, 0, st>>>(reinterpret_cast<const uint4*>(b.o), reinterpret_cast<const uint4*>(b.dout),
-                                            b.lse, b.dl, rows);
+                                            b.lse, b.dl, d.T, d.b, d.L, d.L_src, d.L_ctx, d.T_src, entries);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (d.K_sel < d.T_ctx) {

@@ -1,6 +1,6 @@
 /*
- * isa.h -- C interface of the In-context Sparse Attention (ISA) forward pass
- * for NVIDIA B200 (sm_100a).
+ * isa.h -- C interface of the In-context Sparse Attention (ISA) forward and
+ * backward passes for NVIDIA B200 (sm_100a).
  *
  * The method is the sparse attention of "LIVEditor-14B: Lightning Unified
  * Video Editing via In-Context Sparse Attention" (arXiv:2605.04569), as the
@@ -159,8 +159,9 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
 isa_status isa_forward_static(const isa_params* p, const void* q, const void* k, const void* v, void* out,
                               float* lse, void* stream);
 
-/* Workspace of isa_backward: (lse * log2 e, rowsum(dout * out)) per query
- * row (8 bytes each) and fp32 gradients of the pooled keys and values
+/* Workspace of isa_backward: (lse * log2 e, rowsum(dout * out)) for every
+ * row of every block, padded to `block` rows per block (B*H * T * block * 8
+ * bytes), and fp32 gradients of the pooled keys and values
  * (2 * B*H * T_kv_pad * D * 4 bytes), each 256-byte aligned. */
 isa_status isa_backward_workspace_size(const isa_params* p, size_t* bytes);
 

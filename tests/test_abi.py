@@ -162,10 +162,10 @@ def test_backward_arguments_rejected_before_launch(isa):
     p = isa.make_params(1, 2, 64, 300, 100)
     n = isa.workspace_size(p)
     nb = isa.backward_workspace_size(p)
-    BH, L, T_kv_pad = 2, 400, 128
-    # (lse*log2e, Delta) per row, then dKc and dVc in fp32, each 256-byte aligned
+    BH, T, b, T_kv_pad = 2, 5 + 2, 64, 128
+    # (lse*log2e, Delta) per padded block row, then dKc and dVc in fp32, each 256-byte aligned
     a256 = lambda x: (x + 255) // 256 * 256
-    assert nb == a256(BH * L * 8) + 2 * a256(BH * T_kv_pad * 64 * 4)
+    assert nb == a256(BH * T * b * 8) + 2 * a256(BH * T_kv_pad * 64 * 4)
     a = 1 << 20
     args = [ctypes.byref(p), a, a, a, a, n, a, a, a, a, a, a, a, nb, None]
 
