@@ -9,4 +9,5 @@ from .isa_oracle import (Params, HeadPlan, segment_blocks, pool, coarse_scores,
                          split_sharp_flat, plan_head, forward_head, dense_attention,
                          isa_forward, n_select, n_flat_blocks, n_exact_blocks,
                          sharp_block, flat_block, rope_decoupled,
-                         backward_head, isa_backward)
+                         backward_head, isa_backward, coarse_output,
+                         coarse_residual, coarse_residual_backward)

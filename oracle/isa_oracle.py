@@ -25,7 +25,8 @@ The oracle follows the steps in the order of [R] "Method steps in detail":
       with the highest coarse score is attended exactly; every other kept
       block contributes exp(q Kc_j^T / sqrt(D)) * Vc_j weighted by its token
       count; one softmax normaliser over both parts
-  (6) outputs return to token order (no gamma * O_coarse residual).
+  (6) outputs return to token order; the gamma * O_coarse residual is a
+      separate add-on (``coarse_residual``, reading above its definition).
 The backward (``backward_head``, ``isa_backward``) differentiates steps
 (4)-(6) with the plan held fixed; see the note above ``backward_head``.
 
@@ -488,3 +489,57 @@ def isa_backward(q, k, v, dout, p: Params):
     if single:
         out = [x[0] for x in out]
     return tuple(out)
+
+
+# ----------------------------------------------------------------------------
+# step (6): gamma * O_coarse low-frequency residual
+# ----------------------------------------------------------------------------
+# [R] step (6) adds gamma * O_coarse to the scattered output as a
+# low-frequency residual without defining either.  Reading: O_coarse is the
+# output of the block-level (pooling) attention the method already computes
+# in step (1) -- [R] "Block-sparse attention and pooling attention":
+# attention at low resolution on the pooled means -- i.e. row i of
+# softmax(S) Vc over all T blocks, with S = Qc Kc^T * s the coarse scores;
+# every token of query block i receives gamma * O_coarse_i.  gamma is a
+# scalar the caller supplies (a learned weight in training).
+
+def coarse_output(plan: HeadPlan) -> np.ndarray:
+    """O_coarse [T, D]: softmax over all T blocks of each row of the coarse
+    scores, times the pooled values."""
+    return softmax_rows(plan.S) @ plan.Vc
+
+
+def coarse_residual(plan: HeadPlan, p: Params, gamma: float) -> np.ndarray:
+    """gamma * O_coarse of each token's block, [L, D]."""
+    oc = coarse_output(plan)
+    res = np.zeros((p.L, p.D))
+    for i in range(plan.T):
+        res[plan.starts[i]:plan.starts[i] + plan.counts[i]] = gamma * oc[i]
+    return res
+
+
+def coarse_residual_backward(plan: HeadPlan, p: Params, gamma: float, dout):
+    """Gradients of sum(dout * coarse_residual) with respect to q, k, v
+    ([L, D] each, through the pooled means: 1/n_j per token of block j) and
+    to gamma.  O = P Vc with P = softmax(S), S = s Qc Kc^T."""
+    dout = np.asarray(dout, np.float64)
+    T = plan.T
+    P = softmax_rows(plan.S)
+    oc = P @ plan.Vc
+    dO = np.zeros((T, p.D))
+    for i in range(T):
+        dO[i] = dout[plan.starts[i]:plan.starts[i] + plan.counts[i]].sum(axis=0)
+    dgamma = float((dO * oc).sum())
+    dO *= gamma
+    dP = dO @ plan.Vc.T
+    dS = P * (dP - (dO * oc).sum(axis=1, keepdims=True))
+    dQc = p.s * (dS @ plan.Kc)
+    dKc = p.s * (dS.T @ plan.Qc)
+    dVc = P.T @ dO
+    dq, dk, dv = (np.zeros((p.L, p.D)) for _ in range(3))
+    for j in range(T):
+        t = slice(plan.starts[j], plan.starts[j] + plan.counts[j])
+        dq[t] += dQc[j] / plan.counts[j]
+        dk[t] += dKc[j] / plan.counts[j]
+        dv[t] += dVc[j] / plan.counts[j]
+    return dq, dk, dv, dgamma
