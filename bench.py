@@ -350,6 +350,27 @@ def run_gpu(args, w: Workload):
         # algorithmic work: five products per (query, column) pair against the forward's two
         bwd = {"ms": bwd_ms, "tflops": 2.5 * attn_flops / (bwd_ms / 1e3) / 1e12, "launches_per_call": 5,
                "flops_convention": "2.5 x the forward's attention FLOPs (5 vs 2 matrix products)"}
+        # step (6)'s gamma * O_coarse residual on the same plan (an add-on of
+        # isa_coarse_residual; gamma = 1 for timing)
+        coarse = None
+        if not args.skip_coarse:
+            tmp = out.clone()
+            cws = torch.empty(isa.coarse_residual_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+            for _ in range(2):
+                isa.coarse_residual(tmp, ws, p, 1.0)
+                isa.coarse_residual_backward(ws, p, 1.0, dout, dq, dk, dv, cws=cws)
+            ev4 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev4[0].record(stream)
+            for _ in range(nbk):
+                isa.coarse_residual(tmp, ws, p, 1.0)
+            ev4[1].record(stream)
+            for _ in range(nbk):
+                isa.coarse_residual_backward(ws, p, 1.0, dout, dq, dk, dv, cws=cws)
+            ev4[2].record(stream)
+            torch.cuda.synchronize(dev)
+            coarse = {"forward_ms": ev4[0].elapsed_time(ev4[1]) / nbk, "backward_ms": ev4[1].elapsed_time(ev4[2]) / nbk}
+            del tmp, cws
+        bwd["coarse_residual"] = coarse
         del dout, dq, dk, dv, bws, lse
 
     # end to end through the public API from pinned host memory
@@ -434,6 +455,7 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-coarse", action="store_true")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N>1: replicas = every rank runs the whole workload (weak scaling); "
                          "heads = the ranks split the B*H heads of one workload (strong scaling)")

@@ -14,7 +14,8 @@ Video Editing via In-Context Sparse Attention" (paper.rainbus.top summary,
   forward(...) steps (4)-(6), sharp and flat query blocks in one launch
   backward(...) gradients of steps (4)-(6) with the plan held fixed
   dense(...)   the full attention that ISA replaces
-  IsaAttention torch.autograd.Function over plan + forward / backward
+  coarse_residual(...) step (6)'s gamma * O_coarse residual (and its backward)
+  IsaAttention torch.autograd.Function over plan + forward (+ residual) / backward
 """
 from __future__ import annotations
 
@@ -39,6 +40,7 @@ EXPORTS = (
     "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
     "isa_forward_static", "isa_rope_workspace_size", "isa_rope", "isa_backward_workspace_size", "isa_backward",
+    "isa_coarse_residual", "isa_coarse_residual_backward_workspace_size", "isa_coarse_residual_backward",
 )
 
 
@@ -97,9 +99,13 @@ def load_library() -> ctypes.CDLL:
     lib.isa_rope.argtypes = [P, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]
     lib.isa_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.isa_backward.argtypes = [P, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.isa_coarse_residual.argtypes = [P, ctypes.c_float, vp, sz, vp, vp]
+    lib.isa_coarse_residual_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.isa_coarse_residual_backward.argtypes = [P, ctypes.c_float, vp, sz, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
                  "isa_set_wait_timeout_ns", "isa_set_fault_injection", "isa_rope_workspace_size", "isa_rope",
-                 "isa_backward_workspace_size", "isa_backward"):
+                 "isa_backward_workspace_size", "isa_backward", "isa_coarse_residual",
+                 "isa_coarse_residual_backward_workspace_size", "isa_coarse_residual_backward"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -263,25 +269,67 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ws: torch.Tensor
     return dq, dk, dv
 
 
+def coarse_residual(out: torch.Tensor, ws: torch.Tensor, p: Params, gamma: float, stream=None) -> torch.Tensor:
+    """out += gamma * O_coarse in place (step (6)'s low-frequency residual:
+    block-level softmax(Qc Kc^T s) Vc of the plan in `ws`, broadcast to each
+    token of its query block); returns out."""
+    _check_qkv(out, out, out, p)
+    _check(load_library().isa_coarse_residual(ctypes.byref(p), float(gamma), ws.data_ptr(), ws.numel(),
+                                              out.data_ptr(), _stream(stream)))
+    return out
+
+
+def coarse_residual_backward_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().isa_coarse_residual_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def coarse_residual_backward(ws: torch.Tensor, p: Params, gamma: float, dout: torch.Tensor, dq: torch.Tensor,
+                             dk: torch.Tensor, dv: torch.Tensor, dgamma: Optional[torch.Tensor] = None,
+                             cws: Optional[torch.Tensor] = None, stream=None):
+    """Adds the residual's gradients to dq, dk, dv in place and writes the
+    per-head gradient of gamma to `dgamma` (fp32 [B, H], if given)."""
+    _check_qkv(dq, dk, dv, p)
+    _check_qkv(dout, dout, dout, p)
+    if cws is None:
+        cws = torch.empty(coarse_residual_backward_workspace_size(p), dtype=torch.uint8, device=dq.device)
+    if dgamma is not None and (dgamma.dtype != torch.float32 or dgamma.numel() != p.B * p.H or not dgamma.is_cuda):
+        raise IsaError(ISA_ERR_INVALID_ARG, "dgamma must be a CUDA float32 tensor of B*H elements")
+    _check(load_library().isa_coarse_residual_backward(
+        ctypes.byref(p), float(gamma), ws.data_ptr(), ws.numel(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), dgamma.data_ptr() if dgamma is not None else None, cws.data_ptr(), cws.numel(),
+        _stream(stream)))
+    return dq, dk, dv, dgamma
+
+
 class IsaAttention(torch.autograd.Function):
     """ISA as a differentiable op: forward = plan + sparse attention (keeping
-    the plan, output and lse), backward = the library's backward with that
-    plan.  Inputs are contiguous bf16 CUDA tensors [B, H, L, D]."""
+    the plan, output and lse), plus gamma * O_coarse when gamma != 0;
+    backward = the library's backward with that plan (and the residual's).
+    Call as IsaAttention.apply(q, k, v, p, gamma); inputs are contiguous
+    bf16 CUDA tensors [B, H, L, D]; gamma is a constant (0.0: no residual;
+    its gradient is available from coarse_residual_backward)."""
 
     @staticmethod
-    def forward(ctx, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params) -> torch.Tensor:
+    def forward(ctx, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, gamma: float):
         ws = plan(q, k, v, p)
         lse = torch.empty(p.B, p.H, p.L_src + p.L_ctx, dtype=torch.float32, device=q.device)
         out = forward(q, k, v, ws, p, lse=lse)
         ctx.save_for_backward(q, k, v, ws, out, lse)
-        ctx.p = p
+        ctx.p, ctx.gamma = p, float(gamma)
+        if gamma != 0.0:
+            return coarse_residual(out.clone(), ws, p, gamma)
         return out
 
     @staticmethod
     def backward(ctx, dout: torch.Tensor):
         q, k, v, ws, out, lse = ctx.saved_tensors
-        dq, dk, dv = backward(q, k, v, ws, ctx.p, out, lse, dout.contiguous())
-        return dq, dk, dv, None
+        dout = dout.contiguous()
+        dq, dk, dv = backward(q, k, v, ws, ctx.p, out, lse, dout)
+        if ctx.gamma != 0.0:
+            coarse_residual_backward(ws, ctx.p, ctx.gamma, dout, dq, dk, dv)
+        return dq, dk, dv, None, None
 
 
 def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,

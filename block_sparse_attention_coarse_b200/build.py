@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu", "isa_rope.cu", "isa_bwd.cu"]
+SOURCES = ["isa_api.cu", "isa_plan.cu", "isa_attn.cu", "isa_static.cu", "isa_rope.cu", "isa_bwd.cu", "isa_coarse.cu"]
 LIB = os.path.join(HERE, "libisa.so")
 HEADERS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(ROOT, "include", "isa.h")]

@@ -452,6 +452,56 @@ isa_status isa_backward(const isa_params* p, const void* q, const void* k, const
   return ISA_OK;
 }
 
+isa_status isa_coarse_residual(const isa_params* p, float gamma, const void* ws, size_t ws_bytes, void* out,
+                               void* stream) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if (!std::isfinite(gamma)) return fail(ISA_ERR_INVALID_ARG, "gamma must be finite");
+  if ((s = check_ptr(ws, "workspace", 256)) != ISA_OK || (s = check_ptr(out, "out", 16)) != ISA_OK) return s;
+  const PlanLayout L = make_layout(d);
+  if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  if ((s = bind_device_of(out, "out")) != ISA_OK) return s;
+  const PlanPtrs pp = make_ptrs(L, const_cast<void*>(ws));
+  cudaError_t e = launch_coarse(d, pp, gamma, out, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "coarse residual launch");
+  return ISA_OK;
+}
+
+isa_status isa_coarse_residual_backward_workspace_size(const isa_params* p, size_t* bytes) {
+  if (!bytes) return fail(ISA_ERR_INVALID_ARG, "bytes is NULL");
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  *bytes = coarse_backward_bytes(d);
+  return ISA_OK;
+}
+
+isa_status isa_coarse_residual_backward(const isa_params* p, float gamma, const void* ws, size_t ws_bytes,
+                                        const void* dout, void* dq, void* dk, void* dv, float* dgamma, void* cws,
+                                        size_t cws_bytes, void* stream) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if (!std::isfinite(gamma)) return fail(ISA_ERR_INVALID_ARG, "gamma must be finite");
+  if ((s = check_ptr(ws, "workspace", 256)) != ISA_OK || (s = check_ptr(dout, "dout", 16)) != ISA_OK ||
+      (s = check_ptr(dq, "dq", 16)) != ISA_OK || (s = check_ptr(dk, "dk", 16)) != ISA_OK ||
+      (s = check_ptr(dv, "dv", 16)) != ISA_OK || (s = check_ptr(cws, "coarse workspace", 256)) != ISA_OK)
+    return s;
+  if (dgamma && (s = check_ptr(dgamma, "dgamma", 4)) != ISA_OK) return s;
+  const PlanLayout L = make_layout(d);
+  if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  const size_t need = coarse_backward_bytes(d);
+  if (cws_bytes < need) return fail(ISA_ERR_WORKSPACE, "coarse workspace has %zu bytes, needs %zu", cws_bytes, need);
+  if ((s = bind_device_of(dq, "dq")) != ISA_OK) return s;
+  const PlanPtrs pp = make_ptrs(L, const_cast<void*>(ws));
+  cudaError_t e = launch_coarse(d, pp, gamma, nullptr, dout, dq, dk, dv, dgamma, cws,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "coarse residual backward launch");
+  return ISA_OK;
+}
+
 isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes) {
   Dims d;
   isa_status s = make_dims(p, &d);

@@ -78,6 +78,9 @@ cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void
 cudaError_t prepare_plan_kernels();
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_backward(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sm_count, cudaStream_t st);
+size_t coarse_backward_bytes(const Dims& d);
+cudaError_t launch_coarse(const Dims& d, const PlanPtrs& pp, float gamma, void* out, const void* dout, void* dq,
+                          void* dk, void* dv, float* dgamma, void* cws, cudaStream_t st);
 size_t rope_table_bytes(const Dims& d);
 cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
                         int sm_count, cudaStream_t st);

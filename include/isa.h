@@ -194,6 +194,36 @@ isa_status isa_backward(const isa_params* p, const void* q, const void* k, const
                         size_t ws_bytes, const void* out, const float* lse, const void* dout, void* dq, void* dk,
                         void* dv, void* bws, size_t bws_bytes, void* stream);
 
+/* Step (6) of "Method steps in detail" adds gamma * O_coarse to the
+ * scattered output as a low-frequency residual; the summary card defines
+ * neither.  Reading: O_coarse is the block-level pooling attention of its
+ * "Block-sparse attention and pooling attention" background on the plan's
+ * pooled means, O_coarse_i = sum_j softmax_j(scale * Qc_i . Kc_j) Vc_j over
+ * all T blocks, and every token of query block i receives gamma * O_coarse_i.
+ *   ws    : a workspace isa_plan filled (its Qc, Kc, Vc are used)
+ *   out   : device bf16 [B,H,L,D]; out += gamma * O_coarse in place (fp32
+ *           arithmetic, one rounding to bf16)
+ *   gamma : finite
+ * Apply it to a copy of isa_forward's output: isa_backward needs the sparse
+ * output itself.  One launch (CUDA cores: T x T x D per head). */
+isa_status isa_coarse_residual(const isa_params* p, float gamma, const void* ws, size_t ws_bytes, void* out,
+                               void* stream);
+
+/* Workspace of isa_coarse_residual_backward: per-block statistics and the
+ * scaled block sums of dout (B*H * T * (8 + 4*D) bytes, 256-byte aligned). */
+isa_status isa_coarse_residual_backward_workspace_size(const isa_params* p, size_t* bytes);
+
+/* Gradients of sum(dout * gamma * O_coarse) (see isa_coarse_residual),
+ * ADDED in place to dq, dk, dv (device bf16 [B,H,L,D], e.g. isa_backward's
+ * results), through the pooled means: a block's gradient reaches each of
+ * its n_j tokens divided by n_j.  dgamma: device fp32 [B*H] receiving
+ * sum(dout * O_coarse) per head (zeroed by the call), or NULL.  cws:
+ * caller-owned scratch of isa_coarse_residual_backward_workspace_size bytes,
+ * 256-byte aligned.  Two launches. */
+isa_status isa_coarse_residual_backward(const isa_params* p, float gamma, const void* ws, size_t ws_bytes,
+                                        const void* dout, void* dq, void* dk, void* dv, float* dgamma, void* cws,
+                                        size_t cws_bytes, void* stream);
+
 /* Workspace of isa_rope: the cos/sin table, max(L_src, L_ctx) * D/2 float
  * pairs (8 bytes each). */
 isa_status isa_rope_workspace_size(const isa_params* p, size_t* bytes);

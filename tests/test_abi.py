@@ -181,3 +181,25 @@ def test_backward_arguments_rejected_before_launch(isa):
     assert call(_12=a + 16) == 1 and b"backward workspace" in lib.isa_last_error()
     assert call(_13=nb - 1) == 3
     assert call(_5=n - 1) == 3
+
+
+def test_coarse_residual_arguments_rejected_before_launch(isa):
+    """isa_coarse_residual(_backward) check gamma, pointers and workspace
+    sizes on the host (fake device addresses: nothing may be launched)."""
+    lib = isa.load_library()
+    p = isa.make_params(1, 2, 64, 300, 100)
+    n = isa.workspace_size(p)
+    nc = ctypes.c_size_t()
+    assert lib.isa_coarse_residual_backward_workspace_size(ctypes.byref(p), ctypes.byref(nc)) == 0
+    BH, T = 2, 5 + 2
+    assert nc.value == (BH * T * 8 + 255) // 256 * 256 + BH * T * 64 * 4
+    a = 1 << 20
+    assert lib.isa_coarse_residual(ctypes.byref(p), float("nan"), a, n, a, None) == 1
+    assert b"gamma" in lib.isa_last_error()
+    assert lib.isa_coarse_residual(ctypes.byref(p), 1.0, a, n - 1, a, None) == 3
+    assert lib.isa_coarse_residual(ctypes.byref(p), 1.0, a, n, a + 4, None) == 1
+    args = [ctypes.byref(p), 1.0, a, n, a, a, a, a, None, a, nc.value, None]
+    assert lib.isa_coarse_residual_backward(*(args[:4] + [None] + args[5:])) == 1
+    assert b"dout is NULL" in lib.isa_last_error()
+    assert lib.isa_coarse_residual_backward(*(args[:10] + [nc.value - 1] + args[11:])) == 3
+    assert lib.isa_coarse_residual_backward(*(args[:8] + [a + 2] + args[9:])) == 1

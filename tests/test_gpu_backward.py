@@ -122,7 +122,7 @@ def test_autograd_function_gradients(isa):
     (gq, gk, gv), _ = run_gpu(isa, w, qb, kb, vb, db)
     q, k, v = (to_torch_bf16(x).requires_grad_(True) for x in (qb, kb, vb))
     p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
-    out = isa.IsaAttention.apply(q, k, v, p)
+    out = isa.IsaAttention.apply(q, k, v, p, 0.0)
     out.backward(to_torch_bf16(db))
     torch.cuda.synchronize()
     for g, t in ((gq, q), (gk, k), (gv, v)):
