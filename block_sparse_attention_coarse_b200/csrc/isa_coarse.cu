@@ -35,80 +35,86 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int kRows = 8;           // most query (key) blocks per CTA
+
+// Lane's D/32 consecutive elements of a D-vector (float4 or float2).
 template <int D>
-__device__ __forceinline__ float warp_dot(const float* __restrict__ a, const float* __restrict__ b) {
-  // D/32 consecutive elements per lane (float4 or float2), reduced over the warp
+struct Frag {
+  float v[D / 32];
+};
+template <int D>
+__device__ __forceinline__ Frag<D> frag(const float* __restrict__ x) {
+  Frag<D> f;
   const int lane = threadIdx.x & 31;
-  float acc = 0.f;
   if constexpr (D == 128) {
-    const float4 x = reinterpret_cast<const float4*>(a)[lane], y = reinterpret_cast<const float4*>(b)[lane];
-    acc = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+    const float4 t = reinterpret_cast<const float4*>(x)[lane];
+    f.v[0] = t.x; f.v[1] = t.y; f.v[2] = t.z; f.v[3] = t.w;
   } else {
-    const float2 x = reinterpret_cast<const float2*>(a)[lane], y = reinterpret_cast<const float2*>(b)[lane];
-    acc = x.x * y.x + x.y * y.y;
+    const float2 t = reinterpret_cast<const float2*>(x)[lane];
+    f.v[0] = t.x; f.v[1] = t.y;
   }
+  return f;
+}
+template <int D>
+__device__ __forceinline__ float fdot(const Frag<D>& a, const Frag<D>& b) {
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc = fmaf(a.v[e], b.v[e], acc);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
   return acc;
 }
 
-// Block-wide max or sum of one value per thread (all threads must call).
-template <bool MAX>
-__device__ __forceinline__ float block_reduce(float v, float* red) {
+// Softmax of rows r < nr of pr[r * ld .. + T) in place (log2-unit scores),
+// one warp per row; lse2[r] receives each row's log2 normaliser.
+__device__ void rows_softmax(float* pr, int ld, int T, int nr, float* lse2) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp < nr) {
+    float* row = pr + (size_t)warp * ld;
+    float m = -INFINITY;
+    for (int j = lane; j < T; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o = __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    v = MAX ? fmaxf(v, o) : v + o;
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    float l = 0.f;
+    for (int j = lane; j < T; j += 32) {
+      const float e = exp2f(row[j] - m);
+      row[j] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
+    const float inv = 1.f / l;
+    for (int j = lane; j < T; j += 32) row[j] *= inv;
+    if (lane == 0) lse2[warp] = m + __log2f(l);
   }
   __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float r = red[0];
-  for (int w = 1; w < kWarps; ++w) r = MAX ? fmaxf(r, red[w]) : r + red[w];
-  return r;
 }
 
-// Row i of P = softmax(s Qc Kc^T) into pr[0..T) (shared), its log2 normaliser
-// returned: scores in log2 units, one warp per key block.
+// out[r][d] = sum_j w[r * ld + j] X[j][d] for r < nr (shared out [kRows][D]):
+// each thread owns one column and a slice of j, with kRows accumulators, so
+// every X row is read once for all nr rows; slices combined through `part`.
 template <int D>
-__device__ float coarse_row(const float* __restrict__ Qc_i, const float* __restrict__ Kc, int T, float sl2,
-                            float* pr, float* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int j = warp; j < T; j += kWarps) {
-    const float d = warp_dot<D>(Qc_i, Kc + (size_t)j * D);
-    if (lane == 0) pr[j] = d * sl2;
-  }
-  __syncthreads();
-  float m = -INFINITY;
-  for (int j = threadIdx.x; j < T; j += kThreads) m = fmaxf(m, pr[j]);
-  m = block_reduce<true>(m, red);
-  float l = 0.f;
-  for (int j = threadIdx.x; j < T; j += kThreads) {
-    const float e = exp2f(pr[j] - m);
-    pr[j] = e;
-    l += e;
-  }
-  l = block_reduce<false>(l, red);
-  const float inv = 1.f / l;
-  for (int j = threadIdx.x; j < T; j += kThreads) pr[j] *= inv;
-  __syncthreads();
-  return m + __log2f(l);
-}
-
-// oc[0..D) = sum_j pr[j] Vc_j (shared), two halves of the threads over j.
-template <int D>
-__device__ void coarse_combine(const float* pr, const float* __restrict__ Vc, int T, float* oc, float* part) {
-  constexpr int SPLIT = kThreads / D;   // 2 (D=128) or 4 (D=64) partial sums per column
+__device__ void rows_combine(const float* w, int ld, int nr, const float* __restrict__ X, int T, float* out,
+                             float* part) {
+  constexpr int SPLIT = kThreads / D;
   const int d = threadIdx.x % D, h = threadIdx.x / D;
-  float acc = 0.f;
-  for (int j = h; j < T; j += SPLIT) acc = fmaf(pr[j], Vc[(size_t)j * D + d], acc);
-  part[threadIdx.x] = acc;
+  float acc[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
+  for (int j = h; j < T; j += SPLIT) {
+    const float x = X[(size_t)j * D + d];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (r < nr) acc[r] = fmaf(w[(size_t)r * ld + j], x, acc[r]);
+  }
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) part[(h * kRows + r) * D + d] = acc[r];
   __syncthreads();
-  if (threadIdx.x < D) {
-    float s = 0.f;
-    for (int k = 0; k < SPLIT; ++k) s += part[k * D + threadIdx.x];
-    oc[threadIdx.x] = s;
+  for (int e = threadIdx.x; e < nr * D; e += kThreads) {
+    const int r = e / D, c = e % D;
+    float sum = 0.f;
+    for (int k = 0; k < SPLIT; ++k) sum += part[(k * kRows + r) * D + c];
+    out[r * D + c] = sum;
   }
   __syncthreads();
 }
@@ -133,6 +139,7 @@ __device__ void add_rows(__nv_bfloat16* x, size_t t0, int n, const float* v, flo
 struct CoarseArgs {
   const float *Qc, *Kc, *Vc;   // plan: [BH, T, D]
   int T, T_src, L, L_src, L_ctx, b;
+  int rows;                    // query (key) blocks per CTA, <= kRows
   float sl2, scale, gamma;
   __nv_bfloat16* out;          // forward: out += gamma * O_coarse
   const __nv_bfloat16* dout;   // backward
@@ -142,138 +149,240 @@ struct CoarseArgs {
   float* dO;                   // [BH, T, D] gamma * block sums of dout
 };
 
+// Shared memory: D-vectors first (read as float4 / float2), then the
+// combine scratch, then the [rows][T] score rows.
+template <int D>
+constexpr int kVecFloats = 2 * kRows * D;
+template <int D>
+constexpr int kPartFloats = (kThreads / D) * kRows * D;
+
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_fwd_kernel(const CoarseArgs a) {
   extern __shared__ __align__(16) float sm[];
-  float* oc = sm;                  // D
-  float* part = oc + D;            // kThreads
-  float* red = part + kThreads;    // kWarps
-  float* pr = red + kWarps;        // T
-  const int bh = blockIdx.x, i = blockIdx.y;
+  float* qs = sm;                          // [kRows][D] Qc rows
+  float* oc = qs + kRows * D;              // [kRows][D] O_coarse rows
+  float* part = oc + kRows * D;            // combine scratch
+  float* lse2 = part + kPartFloats<D>;     // [kRows]
+  float* pr = lse2 + kRows;                // [rows][T]
+  const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
+  const int nr = min(a.rows, a.T - i0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t hb = (size_t)bh * a.T * D;
-  coarse_row<D>(a.Qc + hb + (size_t)i * D, a.Kc + hb, a.T, a.sl2, pr, red);
-  coarse_combine<D>(pr, a.Vc + hb, a.T, oc, part);
-  const int2 sp = block_span(i, a.L_src, a.L_ctx, a.b, a.T_src);
-  add_rows<D>(a.out, (size_t)bh * a.L + sp.x, sp.y, oc, a.gamma);
+  for (int e = threadIdx.x; e < nr * D; e += kThreads) qs[e] = a.Qc[hb + (size_t)i0 * D + e];
+  __syncthreads();
+  Frag<D> q[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r)
+    if (r < nr) q[r] = frag<D>(qs + r * D);
+  // scores: one warp per key block, its Kc row fetched once for all nr rows
+  for (int j = warp; j < a.T; j += kWarps) {
+    const Frag<D> k = frag<D>(a.Kc + hb + (size_t)j * D);
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (r < nr) {
+        const float dd = fdot<D>(q[r], k);
+        if (lane == 0) pr[(size_t)r * a.T + j] = dd * a.sl2;
+      }
+    }
+  }
+  __syncthreads();
+  rows_softmax(pr, a.T, a.T, nr, lse2);
+  rows_combine<D>(pr, a.T, nr, a.Vc + hb, a.T, oc, part);
+  for (int r = 0; r < nr; ++r) {
+    const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
+    add_rows<D>(a.out, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.gamma);
+  }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs a) {
-  // D-sized arrays first: dO is read as float4 / float2 by warp_dot
   extern __shared__ __align__(16) float sm[];
-  float* oc = sm;                  // D: O_i
-  float* dO = oc + D;              // D: gamma * sum of dout rows
-  float* dq = dO + D;              // D
-  float* part = dq + D;            // kThreads
-  float* red = part + kThreads;    // kWarps
-  float* pr = red + kWarps;        // T: P_ij, then dS_ij
-  const int bh = blockIdx.x, i = blockIdx.y;
+  float* dO = sm;                          // [kRows][D] gamma * dout block sums (read as fragments)
+  float* oc = dO + kRows * D;              // [kRows][D] O_coarse rows, then dQc rows
+  float* part = oc + kRows * D;            // combine scratch
+  float* lse2 = part + kPartFloats<D>;     // [kRows]
+  float* pr = lse2 + kRows;                // [rows][T] P, then dS
+  const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
+  const int nr = min(a.rows, a.T - i0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t hb = (size_t)bh * a.T * D;
-  const float lse2 = coarse_row<D>(a.Qc + hb + (size_t)i * D, a.Kc + hb, a.T, a.sl2, pr, red);
-  coarse_combine<D>(pr, a.Vc + hb, a.T, oc, part);
-  // sum of the block's dout rows, one column per thread (split over rows)
-  const int2 sp = block_span(i, a.L_src, a.L_ctx, a.b, a.T_src);
+  // scores and softmax, as in the forward (Qc rows staged in dO's space)
+  for (int e = threadIdx.x; e < nr * D; e += kThreads) dO[e] = a.Qc[hb + (size_t)i0 * D + e];
+  __syncthreads();
+  {
+    Frag<D> q[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (r < nr) q[r] = frag<D>(dO + r * D);
+    for (int j = warp; j < a.T; j += kWarps) {
+      const Frag<D> k = frag<D>(a.Kc + hb + (size_t)j * D);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        if (r < nr) {
+          const float dd = fdot<D>(q[r], k);
+          if (lane == 0) pr[(size_t)r * a.T + j] = dd * a.sl2;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  rows_softmax(pr, a.T, a.T, nr, lse2);
+  rows_combine<D>(pr, a.T, nr, a.Vc + hb, a.T, oc, part);
+  // block sums of dout: thread = column, rows of block i0+r split over the thread slices
   {
     constexpr int SPLIT = kThreads / D;
     const int d = threadIdx.x % D, h = threadIdx.x / D;
-    float acc = 0.f;
-    for (int r = h; r < sp.y; r += SPLIT) acc += __bfloat162float(a.dout[((size_t)bh * a.L + sp.x + r) * D + d]);
-    part[threadIdx.x] = acc;
+    for (int r = 0; r < nr; ++r) {
+      const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
+      float acc = 0.f;
+      for (int t = h; t < sp.y; t += SPLIT) acc += __bfloat162float(a.dout[((size_t)bh * a.L + sp.x + t) * D + d]);
+      part[(h * kRows + r) * D + d] = acc;
+    }
     __syncthreads();
-    if (threadIdx.x < D) {
-      float s = 0.f;
-      for (int k = 0; k < SPLIT; ++k) s += part[k * D + threadIdx.x];
-      dO[threadIdx.x] = s;
+    for (int e = threadIdx.x; e < nr * D; e += kThreads) {
+      const int r = e / D, c = e % D;
+      float sum = 0.f;
+      for (int k = 0; k < SPLIT; ++k) sum += part[(k * kRows + r) * D + c];
+      dO[e] = sum;
     }
     __syncthreads();
   }
-  // dgamma partial = (sum of dout rows) . O_i; then dO *= gamma; Delta = dO . O_i
-  float g = threadIdx.x < D ? dO[threadIdx.x] * oc[threadIdx.x] : 0.f;
-  g = block_reduce<false>(g, red);
-  if (threadIdx.x == 0 && a.dgamma) atomicAdd(a.dgamma + bh, g);
-  if (threadIdx.x < D) dO[threadIdx.x] *= a.gamma;
-  __syncthreads();
-  const float delta = a.gamma * g;
-  if (threadIdx.x == 0) a.stat[(size_t)bh * a.T + i] = make_float2(lse2, delta);
-  if (threadIdx.x < D) a.dO[hb + (size_t)i * D + threadIdx.x] = dO[threadIdx.x];
-  // dS_ij = P_ij (dO . Vc_j - Delta), in place of P_ij
-  for (int j = warp; j < a.T; j += kWarps) {
-    const float dp = warp_dot<D>(dO, a.Vc + hb + (size_t)j * D);
-    if (lane == 0) pr[j] = pr[j] * (dp - delta);
+  // per row: g = (dout sum) . O (dgamma), then dO *= gamma, Delta = gamma g;
+  // one warp per row
+  if (warp < nr) {
+    float g = 0.f;
+    for (int c = lane; c < D; c += 32) g = fmaf(dO[warp * D + c], oc[warp * D + c], g);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) g += __shfl_xor_sync(0xFFFFFFFFu, g, off);
+    for (int c = lane; c < D; c += 32) {
+      const float x = a.gamma * dO[warp * D + c];
+      dO[warp * D + c] = x;
+      a.dO[hb + (size_t)(i0 + warp) * D + c] = x;
+    }
+    if (lane == 0) {
+      a.stat[(size_t)bh * a.T + i0 + warp] = make_float2(lse2[warp], a.gamma * g);
+      if (a.dgamma) atomicAdd(a.dgamma + bh, g);
+      lse2[warp] = a.gamma * g;   // Delta of the row, for the dS pass
+    }
   }
   __syncthreads();
-  // dQc_i = s sum_j dS_ij Kc_j
-  coarse_combine<D>(pr, a.Kc + hb, a.T, dq, part);
-  add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, dq, a.scale / (float)sp.y);
+  // dS_rj = P_rj (dO_r . Vc_j - Delta_r), in place; one warp per key block
+  {
+    Frag<D> g[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (r < nr) g[r] = frag<D>(dO + r * D);
+    for (int j = warp; j < a.T; j += kWarps) {
+      const Frag<D> v = frag<D>(a.Vc + hb + (size_t)j * D);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        if (r < nr) {
+          const float dp = fdot<D>(g[r], v);
+          if (lane == 0) pr[(size_t)r * a.T + j] *= dp - lse2[r];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // dQc_r = s sum_j dS_rj Kc_j  -> dq rows of block i0+r += dQc_r / n
+  rows_combine<D>(pr, a.T, nr, a.Kc + hb, a.T, oc, part);
+  for (int r = 0; r < nr; ++r) {
+    const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
+    add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.scale / (float)sp.y);
+  }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArgs a) {
-  // D-sized arrays first: kc and vc are read as float4 / float2 by warp_dot
   extern __shared__ __align__(16) float sm[];
-  float* kc = sm;                  // D: Kc_j
-  float* vc = kc + D;              // D: Vc_j
-  float* gk = vc + D;              // D
-  float* gv = gk + D;              // D
-  float* part = gv + D;            // kThreads
-  float* pj = part + kThreads;     // T: P_ij over query blocks i
-  float* sj = pj + a.T;            // T: dS_ij
-  const int bh = blockIdx.x, j = blockIdx.y;
+  float* kc = sm;                          // [kRows][D] Kc rows, then dKc rows
+  float* vc = kc + kRows * D;              // [kRows][D] Vc rows, then dVc rows
+  float* part = vc + kRows * D;            // combine scratch
+  float* pj = part + kPartFloats<D>;       // [rows][T] P over query blocks
+  float* sj = pj + (size_t)a.rows * a.T;   // [rows][T] dS
+  const int bh = blockIdx.x, j0 = blockIdx.y * a.rows;
+  const int nr = min(a.rows, a.T - j0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t hb = (size_t)bh * a.T * D;
-  if (threadIdx.x < D) {
-    kc[threadIdx.x] = a.Kc[hb + (size_t)j * D + threadIdx.x];
-    vc[threadIdx.x] = a.Vc[hb + (size_t)j * D + threadIdx.x];
+  for (int e = threadIdx.x; e < nr * D; e += kThreads) {
+    kc[e] = a.Kc[hb + (size_t)j0 * D + e];
+    vc[e] = a.Vc[hb + (size_t)j0 * D + e];
   }
   __syncthreads();
-  for (int i = warp; i < a.T; i += kWarps) {
-    const float s = warp_dot<D>(a.Qc + hb + (size_t)i * D, kc);
-    const float dp = warp_dot<D>(a.dO + hb + (size_t)i * D, vc);
-    if (lane == 0) {
+  {
+    Frag<D> k[kRows], v[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (r < nr) {
+        k[r] = frag<D>(kc + r * D);
+        v[r] = frag<D>(vc + r * D);
+      }
+    // one warp per query block i: its Qc and dO rows fetched once for all nr key blocks
+    for (int i = warp; i < a.T; i += kWarps) {
+      const Frag<D> q = frag<D>(a.Qc + hb + (size_t)i * D);
+      const Frag<D> g = frag<D>(a.dO + hb + (size_t)i * D);
       const float2 st = a.stat[(size_t)bh * a.T + i];
-      const float p = exp2f(s * a.sl2 - st.x);
-      pj[i] = p;
-      sj[i] = p * (dp - st.y);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        if (r < nr) {
+          const float s = fdot<D>(q, k[r]);
+          const float dp = fdot<D>(g, v[r]);
+          if (lane == 0) {
+            const float p = exp2f(s * a.sl2 - st.x);
+            pj[(size_t)r * a.T + i] = p;
+            sj[(size_t)r * a.T + i] = p * (dp - st.y);
+          }
+        }
+      }
     }
   }
   __syncthreads();
-  // dKc_j = s sum_i dS_ij Qc_i, dVc_j = sum_i P_ij dO_i
-  coarse_combine<D>(sj, a.Qc + hb, a.T, gk, part);
-  coarse_combine<D>(pj, a.dO + hb, a.T, gv, part);
-  const int2 sp = block_span(j, a.L_src, a.L_ctx, a.b, a.T_src);
-  add_rows<D>(a.dk, (size_t)bh * a.L + sp.x, sp.y, gk, a.scale / (float)sp.y);
-  add_rows<D>(a.dv, (size_t)bh * a.L + sp.x, sp.y, gv, 1.f / (float)sp.y);
+  // dKc_r = s sum_i dS_ri Qc_i, dVc_r = sum_i P_ri dO_i
+  rows_combine<D>(sj, a.T, nr, a.Qc + hb, a.T, kc, part);
+  rows_combine<D>(pj, a.T, nr, a.dO + hb, a.T, vc, part);
+  for (int r = 0; r < nr; ++r) {
+    const int2 sp = block_span(j0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
+    add_rows<D>(a.dk, (size_t)bh * a.L + sp.x, sp.y, kc + r * D, a.scale / (float)sp.y);
+    add_rows<D>(a.dv, (size_t)bh * a.L + sp.x, sp.y, vc + r * D, 1.f / (float)sp.y);
+  }
 }
 
+// Shared-memory bytes of each kernel for `rows` blocks per CTA.
 template <int D>
-static cudaError_t launch_t(const Dims& d, const CoarseArgs& a, bool backward, cudaStream_t st) {
-  const dim3 grid(d.BH, d.T);
-  if (!backward) {
-    const size_t sm = (size_t)(d.T + D + kThreads + kWarps) * 4;
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    coarse_fwd_kernel<D><<<grid, kThreads, sm, st>>>(a);
-    return cudaGetLastError();
-  }
+size_t fwd_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + kRows + (size_t)rows * T) * 4; }
+template <int D>
+size_t kv_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + 2 * (size_t)rows * T) * 4; }
+
+constexpr size_t kSmemBudget = 160 * 1024;
+
+template <int D>
+static cudaError_t launch_t(const Dims& d, CoarseArgs a, bool backward, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+      e = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const size_t smq = (size_t)(d.T + 3 * D + kThreads + kWarps) * 4;
-  coarse_bwd_q_kernel<D><<<grid, kThreads, smq, st>>>(a);
+  // as many blocks per CTA as the score rows leave room for (at most kRows)
+  int rq = kRows;
+  while (rq > 1 && fwd_smem<D>(d.T, rq) > kSmemBudget) --rq;
+  a.rows = rq;
+  const dim3 gq(d.BH, (d.T + rq - 1) / rq);
+  if (!backward) {
+    coarse_fwd_kernel<D><<<gq, kThreads, fwd_smem<D>(d.T, rq), st>>>(a);
+    return cudaGetLastError();
+  }
+  coarse_bwd_q_kernel<D><<<gq, kThreads, fwd_smem<D>(d.T, rq), st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smk = (size_t)(4 * D + 2 * d.T + kThreads) * 4;
-  coarse_bwd_kv_kernel<D><<<grid, kThreads, smk, st>>>(a);
+  int rk = kRows;
+  while (rk > 1 && kv_smem<D>(d.T, rk) > kSmemBudget) --rk;
+  a.rows = rk;
+  coarse_bwd_kv_kernel<D><<<dim3(d.BH, (d.T + rk - 1) / rk), kThreads, kv_smem<D>(d.T, rk), st>>>(a);
   return cudaGetLastError();
 }
 
