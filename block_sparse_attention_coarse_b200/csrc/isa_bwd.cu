@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const AttnArgs& a = b.a;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t kv_full, kv_empty, q_full[kNSQ], q_empty[kNSQ], sd_full[2], ds_full[2];
-  __shared__ __align__(8) uint64_t acc_ready, acc_free, drain_bar;
+  __shared__ __align__(8) uint64_t acc_ready, acc_free, drain_bar, inject_bar;
   __shared__ StepMeta meta[kNSQ];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     mbar_init(&acc_ready, 1);
     mbar_init(&acc_free, 32 * kKvSoft);
     mbar_init(&drain_bar, 1);
+    mbar_init(&inject_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -389,6 +390,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     bool issued = false, ok = true;
+    if (a.inject) ok = warp_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
     int u = 0, n = 0;
     const uint64_t kdesc = smem_desc_sw128(sbase + C::K_OFF, 16, 1024);
     const uint64_t vdesc = smem_desc_sw128(sbase + C::V_OFF, 16, 1024);
@@ -650,7 +652,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const AttnArgs& a = b.a;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[kQNSK], k_empty[kQNSK], v_full[kQNSV], v_empty[kQNSV];
-  __shared__ __align__(8) uint64_t sd_full[2], dp_free, ds_full[2], dq_ready, dq_free, drain_bar;
+  __shared__ __align__(8) uint64_t sd_full[2], dp_free, ds_full[2], dq_ready, dq_free, drain_bar, inject_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -677,6 +679,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     mbar_init(&dq_ready, 1);
     mbar_init(&dq_free, 256);
     mbar_init(&drain_bar, 1);
+    mbar_init(&inject_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -748,6 +751,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     bool issued = false, ok = true;
+    if (a.inject) ok = warp_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
     int n = 0, t0 = 0;
     const uint64_t qdesc = smem_desc_sw128(sbase + C::Q_OFF, 16, 1024);
     const uint64_t odesc = smem_desc_sw128(sbase + C::DO_OFF, 16, 1024);

@@ -261,8 +261,9 @@ const char* isa_version(void);
 isa_status isa_set_wait_timeout_ns(uint64_t ns);
 
 /* Host-chosen fault injection for tests of the timeout path: mode 1 makes
- * the attention kernels wait on a barrier that nothing arrives on, so the
- * wait runs out; 0 turns it off.  Applies to later launches. */
+ * the attention kernels (forward and backward) wait on a barrier that
+ * nothing arrives on, so the wait runs out; 0 turns it off.  Applies to
+ * later launches. */
 isa_status isa_set_fault_injection(int32_t mode);
 
 #ifdef __cplusplus

@@ -168,3 +168,37 @@ def test_backward_rejects_missing_lse(isa):
     out = isa.forward(q, k, v, ws, p)
     with pytest.raises(isa.IsaError):
         isa.backward(q, k, v, ws, p, out, torch.empty(1, 1, w.L, dtype=torch.float16, device="cuda"), out)
+
+
+def test_backward_timeout_path_reports_status_and_context_survives(isa):
+    """Fault injection makes both backward kernels' MMA warps wait on a
+    barrier nothing arrives on: every wait must run out, the plan's status
+    word must read ISA_ERR_DEVICE_TIMEOUT, and after a new plan the next
+    backward must be correct."""
+    w = Workload("bto", 1, 2, 64, 256, 128, block=64, alpha_s=0.5, alpha_f=0.5, alpha_ns=0.25, seed=84)
+    qb, kb, vb = generate_bits(w)
+    db = generate_dout_bits(w)
+    q, k, v, do = (to_torch_bf16(x) for x in (qb, kb, vb, db))
+    p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+    ws = isa.plan(q, k, v, p)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device="cuda")
+    out = isa.forward(q, k, v, ws, p, lse=lse)
+    torch.cuda.synchronize()
+    assert int(isa.plan_view(p, ws)["status"].item()) == 0
+    isa.set_wait_timeout_ns(2_000_000)
+    isa.set_fault_injection(1)
+    try:
+        isa.backward(q, k, v, ws, p, out, lse, do)
+        torch.cuda.synchronize()
+    finally:
+        isa.set_fault_injection(0)
+        isa.set_wait_timeout_ns(0)
+    assert int(isa.plan_view(p, ws)["status"].item()) == isa.ISA_ERR_DEVICE_TIMEOUT
+    # a new plan clears the status word; the normal path is intact
+    (gq, gk, gv), view = run_gpu(isa, w, qb, kb, vb, db)
+    op = oracle_params(w)
+    for h in range(w.BH):
+        qh, kh, vh, dh = (bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb, db))
+        pl = O.plan_head(qh, kh, vh, op)
+        if plan_identical(pl, view, h):
+            assert_grads_close((gq[h], gk[h], gv[h]), O.backward_head(qh, kh, vh, pl, op, dh), ("bto", h))
