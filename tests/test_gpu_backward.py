@@ -202,3 +202,40 @@ def test_backward_timeout_path_reports_status_and_context_survives(isa):
         pl = O.plan_head(qh, kh, vh, op)
         if plan_identical(pl, view, h):
             assert_grads_close((gq[h], gk[h], gv[h]), O.backward_head(qh, kh, vh, pl, op, dh), ("bto", h))
+
+
+@pytest.mark.parametrize("name", ["long65k_b32", "sweep_L131072_D64"])
+def test_backward_long_sequences(isa, name):
+    """65536 tokens with b=32 (T = 2048 blocks) and 131072 tokens with D=64:
+    for every head the gradient sums of any softmax attention (sum_t dv_t =
+    sum_r dout_r, sum_t dk_t = 0); for two heads the dq rows of sampled sharp
+    and flat blocks against the oracle (a block's dq rows need only that
+    block's row of the backward)."""
+    w = named_workloads()[name]
+    qb, kb, vb = generate_bits(w)
+    db = generate_dout_bits(w)
+    (gq, gk, gv), view = run_gpu(isa, w, qb, kb, vb, db)
+    dsum = bf16_to_f64(db.reshape(w.BH, w.L, w.D)).sum(axis=1)
+    for h in range(w.BH):
+        for g in (gq[h], gk[h], gv[h]):
+            assert not np.isnan(g).any(), h
+        sv = gv[h].astype(np.float64).sum(axis=0)
+        sk = gk[h].astype(np.float64).sum(axis=0)
+        assert np.all(np.abs(sv - dsum[h]) <= 4 * U * np.abs(gv[h]).astype(np.float64).sum(axis=0) + 1e-3), h
+        assert np.all(np.abs(sk) <= 4 * U * np.abs(gk[h]).astype(np.float64).sum(axis=0) + 1e-3), h
+    op = oracle_params(w)
+    checked = 0
+    for h in (0, 23, 37):
+        q, k, v = (bf16_to_f64(x) for x in head_bits(w, h))
+        dh = bf16_to_f64(dout_head_bits(w, h))
+        pl = O.plan_head(q, k, v, op)
+        if not plan_identical(pl, view, h):
+            continue
+        checked += 1
+        blocks = [int(pl.sharp[0]), int(pl.sharp[-1]), int(pl.flat[0]), int(pl.flat[len(pl.flat) // 2])]
+        ref_dq, _, _ = O.backward_head(q, k, v, pl, op, dh, blocks=blocks)
+        rows = np.concatenate([np.arange(pl.starts[i], pl.starts[i] + pl.counts[i]) for i in blocks])
+        e = np.abs(gq[h][rows] - ref_dq[rows])
+        r = ref_dq[rows]
+        assert e.max() <= MAX_REL * np.abs(r).max() and e.mean() <= MEAN_REL * np.sqrt((r ** 2).mean()), (name, h)
+    assert checked >= 2, checked
