@@ -15,7 +15,7 @@
 //   dS = P * (dP - Delta),  dQ = s dS K,  dK = s dS^T Q,  dV = P^T dO.
 //
 // Launches, in stream order:
-//   bwd_prep_kernel        Delta and lse*log2(e) per query row (HBM-bound)
+//   bwd_prep_kernel        Delta and lse*log2(e) per query row, block-padded (HBM-bound)
 //   bwd_zero_unkept_kernel dK = dV = 0 for context blocks the pre-selection dropped
 //   bwd_kv_kernel (pooled) key/value-stationary over the head's pooled rows:
 //                          dKc_j, dVc_j (fp32) from every flat block
@@ -126,9 +126,10 @@ __global__ void __launch_bounds__(128) bwd_zero_unkept_kernel(const int* __restr
 //   S^T = K Q^T, dP^T = V dO^T         (SS, M=128, N=64, K=D)
 //   P^T = 2^(S^T s log2e + w_j - lse2), dS^T = P^T (dP^T - Delta)   (softmax warps)
 //   dV += P^T dO, dK += dS^T Q         (TS: P^T / dS^T read as bf16 from TMEM)
-// Roles (576 threads, one CTA per SM): warp 0 lane 0 TMA producer (the tile,
-// the query/dO steps and their metadata), warp 1 MMA issuer (converged, one
-// elected lane), warps 2..17: warp w owns TMEM lanes 32*(w%4).. and query
+// Roles (576 threads, one CTA per SM): warp 0 producer (the whole warp finds
+// the steps; lane 0 loads the tile, publishes each step's metadata and
+// issues its copies), warp 1 MMA issuer (converged, one elected lane),
+// warps 2..17: warp w owns TMEM lanes 32*(w%4).. and query
 // columns 16*((w-2)/4).. of each step (four warps per lane quarter, so that
 // each scheduler interleaves four of them), and writes the epilogue.
 constexpr int kKvSoft = 16;                      // softmax warps
