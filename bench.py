@@ -240,6 +240,8 @@ def run_gpu(args, w: Workload):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
 
+    # host threads for drawing inputs: the ranks of one node share its cores
+    gen_threads = max(1, (os.cpu_count() or 1) // world)
     # inputs resident in HBM: replicas -> one full copy of the workload per
     # rank (its own seed); heads -> this rank's contiguous slice of the B*H
     # heads of one workload, drawn head by head with the workload's seed
@@ -248,11 +250,11 @@ def run_gpu(args, w: Workload):
         lo, hi = head_range(w.BH, rank, world)
         if hi == lo:
             raise SystemExit(f"--shard heads: {world} ranks for {w.BH} heads leaves rank {rank} without work")
-        qb, kb, vb = (x.reshape(1, hi - lo, w.L, w.D) for x in generate_bits(w, heads=range(lo, hi)))
+        qb, kb, vb = (x.reshape(1, hi - lo, w.L, w.D) for x in generate_bits(w, heads=range(lo, hi), threads=gen_threads))
         B_r, H_r = 1, hi - lo
     else:
         wr = w.replace(seed=w.seed + 100 * rank) if world > 1 else w
-        qb, kb, vb = generate_bits(wr)
+        qb, kb, vb = generate_bits(wr, threads=gen_threads)
         B_r, H_r = w.B, w.H
 
     def to_dev(x):
@@ -328,9 +330,9 @@ def run_gpu(args, w: Workload):
     if not args.skip_backward:
         from workloads import generate_dout_bits
         if args.shard == "heads":
-            db = generate_dout_bits(w, heads=range(lo, hi)).reshape(1, hi - lo, w.L, w.D)
+            db = generate_dout_bits(w, heads=range(lo, hi), threads=gen_threads).reshape(1, hi - lo, w.L, w.D)
         else:
-            db = generate_dout_bits(wr)
+            db = generate_dout_bits(wr, threads=gen_threads)
         dout = to_dev(db)
         lse = torch.empty(B_r, H_r, w.L, dtype=torch.float32, device=dev)
         isa.forward(q, k, v, ws, p, out=out, lse=lse)

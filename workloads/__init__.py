@@ -211,11 +211,11 @@ def dout_head_bits(w: Workload, bh: int) -> np.ndarray:
     return f32_to_bf16_bits(g.standard_normal((w.L, w.D), dtype=np.float32))
 
 
-def generate_dout_bits(w: Workload, heads: Optional[List[int]] = None) -> np.ndarray:
+def generate_dout_bits(w: Workload, heads: Optional[List[int]] = None, threads: Optional[int] = None) -> np.ndarray:
     """dout bits, [B, H, L, D] (heads=None) or [len(heads), L, D]."""
     hs = list(range(w.BH)) if heads is None else list(heads)
     out = np.empty((len(hs), w.L, w.D), np.uint16)
-    with _cf.ThreadPoolExecutor(max_workers=min(len(hs), os.cpu_count() or 1) or 1) as ex:
+    with _cf.ThreadPoolExecutor(max_workers=max(1, min(len(hs), threads or os.cpu_count() or 1))) as ex:
         for i, x in zip(range(len(hs)), ex.map(lambda h: dout_head_bits(w, h), hs)):
             out[i] = x
     return out.reshape(w.B, w.H, w.L, w.D) if heads is None else out
