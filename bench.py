@@ -379,14 +379,15 @@ def run_gpu(args, w: Workload):
     e2e = None
     if not args.skip_e2e:
         qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb))
+        oh = torch.empty_like(qh).pin_memory()   # the caller's pinned result buffer, reused every step
         for _ in range(2):
-            isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev)
+            isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev, out=oh)
         torch.cuda.synchronize(dev)
         ke = max(2, min(args.steps, 5))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(ke):
-            res = isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev)
+            res = isa.isa_attention(qh, kh, vh, p, ws=ws, device=dev, out=oh)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / ke
@@ -397,7 +398,7 @@ def run_gpu(args, w: Workload):
         e2e = {"value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(3 * q.numel() * 2), "d2h_bytes_per_step": int(res.numel() * 2),
                "ms_per_step": e2e_ms}
-        del qh, kh, vh, res
+        del qh, kh, vh, oh, res
 
     if world > 1:
         dist.barrier()

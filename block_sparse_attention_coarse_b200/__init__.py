@@ -332,25 +332,82 @@ class IsaAttention(torch.autograd.Function):
         return dq, dk, dv, None, None
 
 
+_COPY_STREAMS: Dict[int, tuple] = {}
+
+
+def _copy_streams(dev: torch.device):
+    """Host-to-device and device-to-host copy streams of a device (created once)."""
+    if dev.index not in _COPY_STREAMS:
+        _COPY_STREAMS[dev.index] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _COPY_STREAMS[dev.index]
+
+
 def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,
-                  device=None, rope_base: Optional[float] = None) -> torch.Tensor:
+                  device=None, rope_base: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                  chunks: int = 8) -> torch.Tensor:
     """The user-level call: plan + forward, after the decoupled RoPE of q and
-    k when `rope_base` is given.  CUDA inputs stay on the device; CPU inputs
-    (pinned for overlap) are copied in and the output is copied back to a
-    pinned CPU tensor on the current stream."""
+    k when `rope_base` is given.
+
+    CUDA inputs stay on the device (returns a new device tensor).  CPU
+    inputs (pinned, [B, H, L, D] bf16) are processed in `chunks` contiguous
+    slices of the B*H heads -- heads are independent -- so that the copies
+    of one slice overlap the kernels of the others: host-to-device copies
+    on one stream, planning and attention on the current stream,
+    device-to-host copies into `out` (a pinned CPU tensor, allocated if not
+    given) on a third.  The current stream waits for the last copy, so
+    synchronising it makes `out` complete."""
     if q.is_cuda:
         if rope_base is not None:
             q, k = rope(q, k, p, rope_base)
         ws = plan(q, k, v, p, ws)
         return forward(q, k, v, ws, p)
     dev = torch.device(device or "cuda")
-    qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    if rope_base is not None:
-        qd, kd = rope(qd, kd, p, rope_base, inplace=True)
-    ws = plan(qd, kd, vd, p, ws)
-    od = forward(qd, kd, vd, ws, p)
-    out = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
-    out.copy_(od, non_blocking=True)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    BH, L, D = p.B * p.H, p.L_src + p.L_ctx, p.D
+    shape = (p.B, p.H, L, D)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise IsaError(ISA_ERR_INVALID_ARG, f"{name} must be a contiguous CPU bfloat16 {shape} tensor")
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    elif out.is_cuda or out.dtype != torch.bfloat16 or tuple(out.shape) != shape or not out.is_contiguous():
+        raise IsaError(ISA_ERR_INVALID_ARG, f"out must be a contiguous CPU bfloat16 {shape} tensor")
+    n = max(1, min(BH, int(chunks)))
+    bounds = [BH * c // n for c in range(n + 1)]
+    sub = lambda h: make_params(1, h, D, p.L_src, p.L_ctx, p.block, p.alpha_s, p.alpha_f, p.alpha_ns, p.scale)
+    hmax = max(bounds[c + 1] - bounds[c] for c in range(n))
+    if ws is None or ws.numel() < workspace_size(sub(hmax)):
+        ws = alloc_workspace(sub(hmax), dev)
+    h2d, d2h = _copy_streams(dev)
+    compute = torch.cuda.current_stream(dev)
+    q3, k3, v3, o3 = (t.view(BH, L, D) for t in (q, k, v, out))
+    for c in range(n):
+        lo, hi = bounds[c], bounds[c + 1]
+        if hi == lo:
+            continue
+        pc = sub(hi - lo)
+        with torch.cuda.stream(h2d):
+            qd, kd, vd = (t[lo:hi].unsqueeze(0).to(dev, non_blocking=True) for t in (q3, k3, v3))
+            ready = torch.cuda.Event()
+            ready.record(h2d)
+        compute.wait_event(ready)
+        for t in (qd, kd, vd):
+            t.record_stream(compute)
+        with torch.cuda.stream(compute):
+            if rope_base is not None:
+                qd, kd = rope(qd, kd, pc, rope_base, inplace=True)
+            plan(qd, kd, vd, pc, ws)
+            od = forward(qd, kd, vd, ws, pc)
+            done = torch.cuda.Event()
+            done.record(compute)
+        d2h.wait_event(done)
+        od.record_stream(d2h)
+        with torch.cuda.stream(d2h):
+            o3[lo:hi].copy_(od[0], non_blocking=True)
+    copied = torch.cuda.Event()
+    copied.record(d2h)
+    compute.wait_event(copied)
     return out
 
 
