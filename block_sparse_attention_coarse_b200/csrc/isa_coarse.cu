@@ -12,9 +12,9 @@
 //
 // The work is T x T x D per head (a few GFLOP at 32K tokens), so these are
 // CUDA-core kernels, one CTA per (head, block), 256 threads:
-//   coarse_fwd_kernel   scores of block i against all T pooled keys (one warp
-//                       per key, float4 lanes), softmax, O_coarse_i, and the
-//                       read-modify-write of the block's output rows
+//   coarse_fwd_kernel   scores of up to 8 query blocks against all T pooled keys
+//                       (one key per thread), softmax, O_coarse, and the
+//                       read-modify-write of the blocks' output rows
 //   coarse_bwd_q_kernel per query block i: dO_i = gamma * sum of the block's
 //                       dout rows, Delta_i = dO_i . O_i, dS_ij =
 //                       P_ij (dO_i . Vc_j - Delta_i), dQc_i = s sum_j dS_ij Kc_j
@@ -32,38 +32,9 @@ namespace isa {
 namespace coarse {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kRows = 8;           // most query (key) blocks per CTA
-
-// Lane's D/32 consecutive elements of a D-vector (float4 or float2).
-template <int D>
-struct Frag {
-  float v[D / 32];
-};
-template <int D>
-__device__ __forceinline__ Frag<D> frag(const float* __restrict__ x) {
-  Frag<D> f;
-  const int lane = threadIdx.x & 31;
-  if constexpr (D == 128) {
-    const float4 t = reinterpret_cast<const float4*>(x)[lane];
-    f.v[0] = t.x; f.v[1] = t.y; f.v[2] = t.z; f.v[3] = t.w;
-  } else {
-    const float2 t = reinterpret_cast<const float2*>(x)[lane];
-    f.v[0] = t.x; f.v[1] = t.y;
-  }
-  return f;
-}
-template <int D>
-__device__ __forceinline__ float fdot(const Frag<D>& a, const Frag<D>& b) {
-  float acc = 0.f;
-#pragma unroll
-  for (int e = 0; e < D / 32; ++e) acc = fmaf(a.v[e], b.v[e], acc);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-  return acc;
-}
 
 // Softmax of rows r < nr of pr[r * ld .. + T) in place (log2-unit scores),
 // one warp per row; lse2[r] receives each row's log2 normaliser.
@@ -91,21 +62,31 @@ __device__ void rows_softmax(float* pr, int ld, int T, int nr, float* lse2) {
 }
 
 // out[r][d] = sum_j w[r * ld + j] X[j][d] for r < nr (shared out [kRows][D]):
-// each thread owns one column and a slice of j, with kRows accumulators, so
-// every X row is read once for all nr rows; slices combined through `part`.
+// each thread owns one column and a contiguous slice of j, with kRows
+// accumulators, so every X row is read once for all nr rows, and the
+// weights of 4 consecutive j come in one 16-byte broadcast load (ld is a
+// multiple of 4 and w is zero in [T, ld)); slices combined through `part`.
 template <int D>
 __device__ void rows_combine(const float* w, int ld, int nr, const float* __restrict__ X, int T, float* out,
                              float* part) {
   constexpr int SPLIT = kThreads / D;
   const int d = threadIdx.x % D, h = threadIdx.x / D;
+  const int chunk = ((ld / 4 + SPLIT - 1) / SPLIT) * 4;
+  const int j0 = h * chunk, j1 = min(j0 + chunk, ld);
   float acc[kRows];
 #pragma unroll
   for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
-  for (int j = h; j < T; j += SPLIT) {
-    const float x = X[(size_t)j * D + d];
+  for (int j = j0; j < j1; j += 4) {
+    float x[4];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < nr) acc[r] = fmaf(w[(size_t)r * ld + j], x, acc[r]);
+    for (int i = 0; i < 4; ++i) x[i] = (j + i < T) ? X[(size_t)(j + i) * D + d] : 0.f;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (r < nr) {
+        const float4 wv = *reinterpret_cast<const float4*>(w + (size_t)r * ld + j);
+        acc[r] = fmaf(wv.x, x[0], fmaf(wv.y, x[1], fmaf(wv.z, x[2], fmaf(wv.w, x[3], acc[r]))));
+      }
+    }
   }
 #pragma unroll
   for (int r = 0; r < kRows; ++r) part[(h * kRows + r) * D + d] = acc[r];
@@ -117,6 +98,27 @@ __device__ void rows_combine(const float* w, int ld, int nr, const float* __rest
     out[r * D + c] = sum;
   }
   __syncthreads();
+}
+
+// acc[r] = A[r] . x for r < nr: the rows of A in shared memory (read as
+// 16-byte broadcasts: every lane of a warp reads the same address), x one
+// row of global memory per thread.  Threads take different x rows, so no
+// shuffle reduction is needed.
+template <int D>
+__device__ __forceinline__ void row_dots(const float* A, int nr, const float* __restrict__ x, float (&acc)[kRows]) {
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D; c += 4) {
+    const float4 xv = *reinterpret_cast<const float4*>(x + c);
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (r < nr) {
+        const float4 av = *reinterpret_cast<const float4*>(A + r * D + c);
+        acc[r] = fmaf(av.x, xv.x, fmaf(av.y, xv.y, fmaf(av.z, xv.z, fmaf(av.w, xv.w, acc[r]))));
+      }
+    }
+  }
 }
 
 // rows [t0, t0+n) of x (bf16 [.., D]) += scale * v (shared fp32 [D])
@@ -163,31 +165,24 @@ __global__ void __launch_bounds__(kThreads) coarse_fwd_kernel(const CoarseArgs a
   float* oc = qs + kRows * D;              // [kRows][D] O_coarse rows
   float* part = oc + kRows * D;            // combine scratch
   float* lse2 = part + kPartFloats<D>;     // [kRows]
-  float* pr = lse2 + kRows;                // [rows][T]
+  float* pr = lse2 + kRows;                // [rows][ld], zero past T
   const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
   const int nr = min(a.rows, a.T - i0);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ld = (a.T + 3) & ~3;
   const size_t hb = (size_t)bh * a.T * D;
   for (int e = threadIdx.x; e < nr * D; e += kThreads) qs[e] = a.Qc[hb + (size_t)i0 * D + e];
   __syncthreads();
-  Frag<D> q[kRows];
+  // scores: one key block per thread, against all nr query rows
+  for (int j = threadIdx.x; j < ld; j += kThreads) {
+    float acc[kRows];
+    if (j < a.T) row_dots<D>(qs, nr, a.Kc + hb + (size_t)j * D, acc);
 #pragma unroll
-  for (int r = 0; r < kRows; ++r)
-    if (r < nr) q[r] = frag<D>(qs + r * D);
-  // scores: one warp per key block, its Kc row fetched once for all nr rows
-  for (int j = warp; j < a.T; j += kWarps) {
-    const Frag<D> k = frag<D>(a.Kc + hb + (size_t)j * D);
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      if (r < nr) {
-        const float dd = fdot<D>(q[r], k);
-        if (lane == 0) pr[(size_t)r * a.T + j] = dd * a.sl2;
-      }
-    }
+    for (int r = 0; r < kRows; ++r)
+      if (r < nr) pr[(size_t)r * ld + j] = j < a.T ? acc[r] * a.sl2 : 0.f;
   }
   __syncthreads();
-  rows_softmax(pr, a.T, a.T, nr, lse2);
-  rows_combine<D>(pr, a.T, nr, a.Vc + hb, a.T, oc, part);
+  rows_softmax(pr, ld, a.T, nr, lse2);
+  rows_combine<D>(pr, ld, nr, a.Vc + hb, a.T, oc, part);
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
     add_rows<D>(a.out, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.gamma);
@@ -201,33 +196,25 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs
   float* oc = dO + kRows * D;              // [kRows][D] O_coarse rows, then dQc rows
   float* part = oc + kRows * D;            // combine scratch
   float* lse2 = part + kPartFloats<D>;     // [kRows]
-  float* pr = lse2 + kRows;                // [rows][T] P, then dS
+  float* pr = lse2 + kRows;                // [rows][ld] P, then dS; zero past T
   const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
   const int nr = min(a.rows, a.T - i0);
+  const int ld = (a.T + 3) & ~3;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t hb = (size_t)bh * a.T * D;
   // scores and softmax, as in the forward (Qc rows staged in dO's space)
   for (int e = threadIdx.x; e < nr * D; e += kThreads) dO[e] = a.Qc[hb + (size_t)i0 * D + e];
   __syncthreads();
-  {
-    Frag<D> q[kRows];
+  for (int j = threadIdx.x; j < ld; j += kThreads) {
+    float acc[kRows];
+    if (j < a.T) row_dots<D>(dO, nr, a.Kc + hb + (size_t)j * D, acc);
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
-      if (r < nr) q[r] = frag<D>(dO + r * D);
-    for (int j = warp; j < a.T; j += kWarps) {
-      const Frag<D> k = frag<D>(a.Kc + hb + (size_t)j * D);
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        if (r < nr) {
-          const float dd = fdot<D>(q[r], k);
-          if (lane == 0) pr[(size_t)r * a.T + j] = dd * a.sl2;
-        }
-      }
-    }
+      if (r < nr) pr[(size_t)r * ld + j] = j < a.T ? acc[r] * a.sl2 : 0.f;
   }
   __syncthreads();
-  rows_softmax(pr, a.T, a.T, nr, lse2);
-  rows_combine<D>(pr, a.T, nr, a.Vc + hb, a.T, oc, part);
+  rows_softmax(pr, ld, a.T, nr, lse2);
+  rows_combine<D>(pr, ld, nr, a.Vc + hb, a.T, oc, part);
   // block sums of dout: thread = column, rows of block i0+r split over the thread slices
   {
     constexpr int SPLIT = kThreads / D;
@@ -266,26 +253,17 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs
     }
   }
   __syncthreads();
-  // dS_rj = P_rj (dO_r . Vc_j - Delta_r), in place; one warp per key block
-  {
-    Frag<D> g[kRows];
+  // dS_rj = P_rj (dO_r . Vc_j - Delta_r), in place; one key block per thread
+  for (int j = threadIdx.x; j < a.T; j += kThreads) {
+    float dp[kRows];
+    row_dots<D>(dO, nr, a.Vc + hb + (size_t)j * D, dp);
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
-      if (r < nr) g[r] = frag<D>(dO + r * D);
-    for (int j = warp; j < a.T; j += kWarps) {
-      const Frag<D> v = frag<D>(a.Vc + hb + (size_t)j * D);
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        if (r < nr) {
-          const float dp = fdot<D>(g[r], v);
-          if (lane == 0) pr[(size_t)r * a.T + j] *= dp - lse2[r];
-        }
-      }
-    }
+      if (r < nr) pr[(size_t)r * ld + j] *= dp[r] - lse2[r];
   }
   __syncthreads();
   // dQc_r = s sum_j dS_rj Kc_j  -> dq rows of block i0+r += dQc_r / n
-  rows_combine<D>(pr, a.T, nr, a.Kc + hb, a.T, oc, part);
+  rows_combine<D>(pr, ld, nr, a.Kc + hb, a.T, oc, part);
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
     add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.scale / (float)sp.y);
@@ -298,48 +276,39 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
   float* kc = sm;                          // [kRows][D] Kc rows, then dKc rows
   float* vc = kc + kRows * D;              // [kRows][D] Vc rows, then dVc rows
   float* part = vc + kRows * D;            // combine scratch
-  float* pj = part + kPartFloats<D>;       // [rows][T] P over query blocks
-  float* sj = pj + (size_t)a.rows * a.T;   // [rows][T] dS
+  const int ld = (a.T + 3) & ~3;
+  float* pj = part + kPartFloats<D>;       // [rows][ld] P over query blocks, zero past T
+  float* sj = pj + (size_t)a.rows * ld;    // [rows][ld] dS, zero past T
   const int bh = blockIdx.x, j0 = blockIdx.y * a.rows;
   const int nr = min(a.rows, a.T - j0);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t hb = (size_t)bh * a.T * D;
   for (int e = threadIdx.x; e < nr * D; e += kThreads) {
     kc[e] = a.Kc[hb + (size_t)j0 * D + e];
     vc[e] = a.Vc[hb + (size_t)j0 * D + e];
   }
   __syncthreads();
-  {
-    Frag<D> k[kRows], v[kRows];
+  // one query block per thread: its Qc and dO rows against all nr key blocks
+  for (int i = threadIdx.x; i < ld; i += kThreads) {
+    float s[kRows], dp[kRows];
+    float2 st = make_float2(0.f, 0.f);
+    if (i < a.T) {
+      row_dots<D>(kc, nr, a.Qc + hb + (size_t)i * D, s);
+      row_dots<D>(vc, nr, a.dO + hb + (size_t)i * D, dp);
+      st = a.stat[(size_t)bh * a.T + i];
+    }
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
+    for (int r = 0; r < kRows; ++r) {
       if (r < nr) {
-        k[r] = frag<D>(kc + r * D);
-        v[r] = frag<D>(vc + r * D);
-      }
-    // one warp per query block i: its Qc and dO rows fetched once for all nr key blocks
-    for (int i = warp; i < a.T; i += kWarps) {
-      const Frag<D> q = frag<D>(a.Qc + hb + (size_t)i * D);
-      const Frag<D> g = frag<D>(a.dO + hb + (size_t)i * D);
-      const float2 st = a.stat[(size_t)bh * a.T + i];
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        if (r < nr) {
-          const float s = fdot<D>(q, k[r]);
-          const float dp = fdot<D>(g, v[r]);
-          if (lane == 0) {
-            const float p = exp2f(s * a.sl2 - st.x);
-            pj[(size_t)r * a.T + i] = p;
-            sj[(size_t)r * a.T + i] = p * (dp - st.y);
-          }
-        }
+        const float p = i < a.T ? exp2f(s[r] * a.sl2 - st.x) : 0.f;
+        pj[(size_t)r * ld + i] = p;
+        sj[(size_t)r * ld + i] = i < a.T ? p * (dp[r] - st.y) : 0.f;
       }
     }
   }
   __syncthreads();
   // dKc_r = s sum_i dS_ri Qc_i, dVc_r = sum_i P_ri dO_i
-  rows_combine<D>(sj, a.T, nr, a.Qc + hb, a.T, kc, part);
-  rows_combine<D>(pj, a.T, nr, a.dO + hb, a.T, vc, part);
+  rows_combine<D>(sj, ld, nr, a.Qc + hb, a.T, kc, part);
+  rows_combine<D>(pj, ld, nr, a.dO + hb, a.T, vc, part);
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(j0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
     add_rows<D>(a.dk, (size_t)bh * a.L + sp.x, sp.y, kc + r * D, a.scale / (float)sp.y);
@@ -349,9 +318,9 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
 
 // Shared-memory bytes of each kernel for `rows` blocks per CTA.
 template <int D>
-size_t fwd_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + kRows + (size_t)rows * T) * 4; }
+size_t fwd_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + kRows + (size_t)rows * ((T + 3) & ~3)) * 4; }
 template <int D>
-size_t kv_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + 2 * (size_t)rows * T) * 4; }
+size_t kv_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + 2 * (size_t)rows * ((T + 3) & ~3)) * 4; }
 
 constexpr size_t kSmemBudget = 160 * 1024;
 
