@@ -106,3 +106,26 @@ def test_residual_full_size_sampled_heads(isa):
     for h in (5, 66):
         qh, kh, vh = (bf16_to_f64(x) for x in head_bits(w, h))
         assert_close(got[h], O.coarse_residual(O.plan_head(qh, kh, vh, op), op, 1.0), ("dit14b", h))
+
+
+def test_residual_backward_full_size_sampled_heads(isa):
+    """The bench shape: every element of dq, dk, dv and dgamma of two heads."""
+    w = named_workloads()["dit14b"]
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    do = to_torch_bf16(generate_dout_bits(w))
+    p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block)
+    ws = isa.plan(q, k, v, p)
+    zq, zk, zv = (torch.zeros_like(q) for _ in range(3))
+    dgamma = torch.zeros(w.BH, dtype=torch.float32, device="cuda")
+    isa.coarse_residual_backward(ws, p, 0.75, do, zq, zk, zv, dgamma)
+    torch.cuda.synchronize()
+    op = oracle_params(w)
+    dob = generate_dout_bits(w, heads=[7, 48])
+    for idx, h in enumerate((7, 48)):
+        qh, kh, vh = (bf16_to_f64(x) for x in head_bits(w, h))
+        pl = O.plan_head(qh, kh, vh, op)
+        rq, rk, rv, rg = O.coarse_residual_backward(pl, op, 0.75, bf16_to_f64(dob[idx]))
+        for nm, t, r in (("dq", zq, rq), ("dk", zk, rk), ("dv", zv, rv)):
+            assert_close(t.reshape(w.BH, w.L, w.D)[h].float().cpu().numpy(), r, ("dit14b", h, nm))
+        assert abs(float(dgamma[h]) - rg) <= 1e-4 * max(1.0, abs(rg))
