@@ -181,7 +181,16 @@ class ClockSampler:
                  "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.2)
+        # nvidia-smi takes a moment to start: wait (at most 3 s) for its first
+        # sample so that the timed region is sampled from its start
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 3.0:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    break
+            except OSError:
+                break
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
