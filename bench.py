@@ -17,6 +17,9 @@ collective: by default every rank runs its own copy of the workload (weak
 scaling); `--shard heads` splits the B*H heads of one workload across the
 ranks (strong scaling).  Timing is the max over ranks.
 
+At N=1 the line also carries `long_context`: the same forward step at
+131072 tokens (B=1, H=40, D=128), the metric's second length.
+
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload (rank 0 only).
 """
@@ -234,6 +237,44 @@ class ClockSampler:
 # GPU arm
 # ----------------------------------------------------------------------------
 
+def measure_long(isa, dev, stream, name: str = "sweep_L131072_D128", steps: int = 5, warmup: int = 3) -> dict:
+    """The forward step at the metric's second length, 131072 tokens
+    (B=1, H=40, D=128, b=64, default ratios): plan and attention latency,
+    executed TF/s and the attention kernel's fraction of the measured
+    sustained bf16 peak, CUDA events on `stream`."""
+    import torch
+    w = named_workloads()[name]
+    q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in generate_bits(w))
+    p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+    ws = isa.alloc_workspace(p, dev)
+    out = torch.empty_like(q)
+    for _ in range(warmup):
+        isa.plan(q, k, v, p, ws)
+        isa.forward(q, k, v, ws, p, out=out)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(stream)
+        isa.plan(q, k, v, p, ws)
+        ev[i][1].record(stream)
+        isa.forward(q, k, v, ws, p, out=out)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    view = isa.plan_view(p, ws)
+    flops = isa.executed_flops(p, view)
+    attn_flops = flops - 2.0 * view["T"] ** 2 * w.D * w.BH
+    plan_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps))
+    fwd_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps))
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    res = {"workload": describe(w)["workload"], "plan_ms": plan_ms, "forward_ms": fwd_ms,
+           "ms_per_step": plan_ms + fwd_ms, "value": flops / ((plan_ms + fwd_ms) / 1e3) / 1e12, "unit": "TFLOP/s",
+           "attention_frac": attn_flops / (fwd_ms / 1e3) / 1e12 / peak, "device_status": int(view["status"].item())}
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args, w: Workload):
     import torch
     import torch.distributed as dist
@@ -409,6 +450,11 @@ def run_gpu(args, w: Workload):
                "ms_per_step": e2e_ms}
         del qh, kh, vh, oh, res
 
+    # the metric's second length (131072 tokens), single GPU only
+    long_ctx = None
+    if world == 1 and not args.skip_long and w.name != "sweep_L131072_D128":
+        long_ctx = measure_long(isa, dev, stream)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -448,6 +494,8 @@ def run_gpu(args, w: Workload):
         line["e2e"] = e2e
     if bwd:
         line["backward"] = bwd
+    if long_ctx:
+        line["long_context"] = long_ctx
     if world == 1 and not args.skip_cpu:
         fl, secs, desc = oracle_sample(w)
         line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
@@ -468,6 +516,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-coarse", action="store_true")
+    ap.add_argument("--skip-long", action="store_true", help="skip the 131072-token forward leg")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N>1: replicas = every rank runs the whole workload (weak scaling); "
                          "heads = the ranks split the B*H heads of one workload (strong scaling)")
