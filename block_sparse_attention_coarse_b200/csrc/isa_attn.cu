@@ -460,12 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int R>
 static cudaError_t launch_t(const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st) {
   using C = Cfg<D, R>;
-  static bool attr_done = false;   // per template instance; set once per process
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};   // per template instance
+  cudaError_t e = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(attn_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  });
+  if (e != cudaSuccess) return e;
   attn_kernel<D, R><<<grid, kThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
   return cudaGetLastError();
 }

@@ -957,13 +957,15 @@ template <int D, int R>
 static cudaError_t launch_t(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sms, cudaStream_t st) {
   using KC = KvCfg<D, R>;
   using QC = QCfg<D, R>;
-  static bool attr_done = false;   // per template instance; set once per process
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_kv_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KC::SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QC::SMEM);
+  static std::atomic<unsigned long long> attr_done{0};   // per template instance
+  {
+    const cudaError_t e = once_per_device(attr_done, [] {
+      cudaError_t r = cudaFuncSetAttribute(bwd_kv_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KC::SMEM);
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(bwd_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QC::SMEM);
+      return r;
+    });
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   const size_t entries = (size_t)d.BH * d.T * d.b;
   const int pgrid = (int)std::max<size_t>(1, std::min<size_t>((entries * (D / 8) + 255) / 256, (size_t)sms * 16));

@@ -326,15 +326,17 @@ constexpr size_t kSmemBudget = 160 * 1024;
 
 template <int D>
 static cudaError_t launch_t(const Dims& d, CoarseArgs a, bool backward, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+  static std::atomic<unsigned long long> attr_done{0};   // per template instance
+  {
+    const cudaError_t e = once_per_device(attr_done, [] {
+      cudaError_t r = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+      return r;
+    });
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   // as many blocks per CTA as the score rows leave room for (at most kRows)
   int rq = kRows;

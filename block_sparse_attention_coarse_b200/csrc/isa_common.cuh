@@ -3,6 +3,8 @@
 // tcgen05 MMA / TMEM access) written as inline PTX.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -86,6 +88,22 @@ cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k
                         int sm_count, cudaStream_t st);
 void set_last_error(const char* msg);
 isa_status bind_device_of(const void* ptr, const char* name);
+
+// Kernel attributes (the dynamic shared-memory limit) belong to the module
+// loaded on each device, so they are set on the first launch on every
+// device, not once per process.  `done` holds one bit per device 0..63;
+// devices beyond that set the attributes on every launch.
+template <class F>
+cudaError_t once_per_device(std::atomic<unsigned long long>& done, F&& set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 constexpr int kMaxT = 8192;      // blocks per head
 constexpr int kMaxTkv = 6144;    // kept blocks per head

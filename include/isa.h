@@ -13,9 +13,14 @@
  * split into planning and attention.
  *
  * Conventions shared by every entry point
- *  - Q, K, V and O are bfloat16 tensors [B, H, L, D], contiguous, on the
- *    current CUDA device, with L = L_src + L_ctx and the context tokens
- *    after the source tokens.  Base addresses must be 16-byte aligned.
+ *  - Q, K, V and O are bfloat16 tensors [B, H, L, D], contiguous, on one
+ *    CUDA device, with L = L_src + L_ctx and the context tokens after the
+ *    source tokens.  Base addresses must be 16-byte aligned.
+ *  - Each call runs on the device that holds its tensors: it looks up the
+ *    device of q (of out for isa_coarse_residual, of dq for
+ *    isa_coarse_residual_backward) and makes it the calling thread's
+ *    current device; the stream must belong to that device.  One process
+ *    may so drive several devices, from one host thread or several.
  *  - "device" pointers are CUDA device (or managed) memory; the caller owns
  *    all memory and the stream.  The library allocates no device memory,
  *    launches asynchronously on `stream` (a cudaStream_t, NULL = legacy
