@@ -441,6 +441,7 @@ __device__ inline void warp_topk(const float* key, int n, int k, int* out, uint3
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = t | (1u << bit);
       int c = 0;
+#pragma unroll 4
       for (int i = lane; i < n; i += 32) c += f2ord(key[i]) >= cand;
       c = __reduce_add_sync(0xFFFFFFFFu, c);
       if (c >= k) t = cand;
@@ -448,6 +449,7 @@ __device__ inline void warp_topk(const float* key, int n, int k, int* out, uint3
   }
   int gt = 0;
   if (k > 0) {
+#pragma unroll 4
     for (int i = lane; i < n; i += 32) gt += f2ord(key[i]) > t;
     gt = __reduce_add_sync(0xFFFFFFFFu, gt);
   }

@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(256) ctx_select_kernel(Dims dm, PlanPtrs pp) {
     constexpr int SPLIT = 256 / D;
     const int d = tid % D, part_i = tid / D;
     float s = 0.f;
-    for (int i = part_i; i < dm.T_src; i += SPLIT) s += Qc[(size_t)i * D + d];
+#pragma unroll 16
+    for (int i = part_i; i < dm.T_src; i += SPLIT) s += Qc[(size_t)i * D + d];   // loads in flight, adds in order
     part[tid] = s;
     __syncthreads();
     if (tid < D) {
@@ -96,15 +97,34 @@ __global__ void __launch_bounds__(256) ctx_select_kernel(Dims dm, PlanPtrs pp) {
     __syncthreads();
   }
   const int warp = tid >> 5, lane = tid & 31;
-  for (int c = warp; c < dm.T_ctx; c += 8) {
-    const float* kr = Kc + (size_t)(dm.T_src + c) * D;
-    float s = 0.f;
-    for (int d = lane; d < D; d += 32) s += qsum[d] * kr[d];
+  // four context blocks per warp at a time, so that their Kc rows are
+  // fetched together (each dot product keeps its own order of additions)
+  constexpr int CR = 4, PER = D / 32;
+  for (int c0 = warp * CR; c0 < dm.T_ctx; c0 += 8 * CR) {
+    float kv[CR][PER];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (lane == 0) {
-      imp[c] = s * dm.scale;
-      pp.imp[(size_t)bh * dm.T_ctx + c] = s * dm.scale;
+    for (int u = 0; u < CR; ++u) {
+      const float* kr = Kc + (size_t)(dm.T_src + min(c0 + u, dm.T_ctx - 1)) * D;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) kv[u][e] = kr[lane + 32 * e];
+    }
+    float s[CR];
+#pragma unroll
+    for (int u = 0; u < CR; ++u) {
+      s[u] = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) s[u] += qsum[lane + 32 * e] * kv[u][e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < CR; ++u) s[u] += __shfl_xor_sync(0xFFFFFFFFu, s[u], o);
+    if (lane < CR && c0 + lane < dm.T_ctx) {
+      float v = s[0];
+#pragma unroll
+      for (int u = 1; u < CR; ++u) v = lane == u ? s[u] : v;
+      imp[c0 + lane] = v * dm.scale;
+      pp.imp[(size_t)bh * dm.T_ctx + c0 + lane] = v * dm.scale;
     }
   }
   __syncthreads();
@@ -308,15 +328,35 @@ __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
   constexpr int KS = D + 4;         // padded row stride of the Kc chunk
   float* kch = sc + 8 * dm.T_kv;    // [32][KS]
   const float4* q4 = reinterpret_cast<const float4*>(qrows + warp * D);
+  // Each thread moves NPT float4 of every 32-row chunk: column col4 of rows
+  // r0 + i*RS.  The chunk after the current one is fetched into registers
+  // while the current one is used, and the kept indices one chunk earlier
+  // still, so the two dependent L2 reads overlap the dot products.
+  constexpr int C4 = D / 4, NPT = 32 * C4 / 256, RS = 256 / C4;
+  const int col4 = tid % C4, r0 = tid / C4;
+  int nidx[NPT];
+  float4 w[NPT];
+  auto load_idx = [&](int k) {
+#pragma unroll
+    for (int i = 0; i < NPT; ++i) nidx[i] = k + r0 + i * RS < dm.T_kv ? kept[k + r0 + i * RS] : -1;
+  };
+  auto load_rows = [&]() {
+#pragma unroll
+    for (int i = 0; i < NPT; ++i)
+      w[i] = nidx[i] >= 0 ? reinterpret_cast<const float4*>(Kc + (size_t)nidx[i] * D)[col4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  load_idx(0);
+  load_rows();
+  load_idx(32);
   for (int k0 = 0; k0 < dm.T_kv; k0 += 32) {
     __syncthreads();   // the previous chunk is consumed
-    for (int e = tid; e < 32 * (D / 4); e += 256) {
-      const int r = e / (D / 4), c4 = e % (D / 4);
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k0 + r < dm.T_kv) w = reinterpret_cast<const float4*>(Kc + (size_t)kept[k0 + r] * D)[c4];
-      *reinterpret_cast<float4*>(kch + r * KS + 4 * c4) = w;
-    }
+#pragma unroll
+    for (int i = 0; i < NPT; ++i) *reinterpret_cast<float4*>(kch + (r0 + i * RS) * KS + 4 * col4) = w[i];
     __syncthreads();
+    if (k0 + 32 < dm.T_kv) {
+      load_rows();
+      load_idx(k0 + 64);
+    }
     const float4* k4 = reinterpret_cast<const float4*>(kch + lane * KS);
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll 8
