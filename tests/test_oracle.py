@@ -172,6 +172,11 @@ def test_split_order_and_ties():
     assert sharp.tolist() == [5] and flat.tolist() == [0, 1, 2, 3, 4]
     sharp, flat = O.split_sharp_flat(M, 0)
     assert flat.tolist() == [] and len(sharp) == 6
+    # the boundary inside a tie: of two equal M, the lower block is the sharper
+    sharp, flat = O.split_sharp_flat(M, 4)
+    assert sharp.tolist() == [0, 5] and flat.tolist() == [1, 2, 3, 4]
+    sharp, flat = O.split_sharp_flat(M, 1)
+    assert sharp.tolist() == [0, 1, 2, 3, 5] and flat.tolist() == [4]
 
 
 def test_counts_follow_ratios():
@@ -180,6 +185,26 @@ def test_counts_follow_ratios():
     assert O.n_flat_blocks(0.5, 512) == 256 and O.n_flat_blocks(0.5, 33) == 16
     assert O.n_exact_blocks(0.0625, 288) == 18 and O.n_exact_blocks(0.0625, 210) == 14
     assert O.n_exact_blocks(0.0, 288) == 0 and O.n_exact_blocks(1.0, 288) == 288
+
+
+def test_exact_share_counts_the_kept_blocks():
+    """alpha_ns is a share of the KV blocks the flat path sees, the kept ones
+    (techwalker.com retelling, section 9: alpha_ns = 0.0625 sends 6.25 % of
+    the KV blocks to the exact path and the rest to the Taylor path; the KV
+    set there is the one left after the context pre-selection).  16 + 16
+    tokens in blocks of 2:
+    T_src = T_ctx = 8, alpha_s = 0.25 keeps 2 context blocks, so T_kv = 10
+    and alpha_ns = 0.25 gives ceil(2.5) = 3 exact blocks per flat block (a
+    share of all 16 blocks would give 4).  Exact and pooled blocks split the
+    kept set."""
+    p = O.Params(L_src=16, L_ctx=16, D=4, block=2, alpha_s=0.25, alpha_f=0.5, alpha_ns=0.25)
+    rng = np.random.default_rng(7)
+    q, k, v = (rng.standard_normal((32, 4)) for _ in range(3))
+    pl = O.plan_head(q, k, v, p)
+    assert len(pl.kept) == 10 and len(pl.flat) == 8
+    assert pl.exact.shape == (8, 3)
+    for row in pl.exact:
+        assert len(set(row.tolist())) == 3 and all(0 <= x < 10 for x in row)
 
 
 # ----------------------------------------------------------------------------
