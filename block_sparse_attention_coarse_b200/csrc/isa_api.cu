@@ -15,8 +15,9 @@ using namespace isa;
 namespace {
 
 thread_local std::string g_last_error = "no error";
-uint64_t g_timeout_ns = kDefaultTimeoutNs;
-int g_inject = 0;
+// process-wide settings, read by every launch (any host thread may set them)
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_inject{0};
 
 isa_status fail(isa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 isa_status fail(isa_status s, const char* fmt, ...) {
@@ -310,8 +311,8 @@ static AttnArgs attn_args(const Dims& d, int mode, const PlanPtrs* pp) {
     a.bits = pp->bits;
     a.ctx_sel = pp->ctx_sel;
   }
-  a.timeout_ns = g_timeout_ns;
-  a.inject = g_inject;
+  a.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  a.inject = g_inject.load(std::memory_order_relaxed);
   return a;
 }
 
@@ -534,13 +535,13 @@ const char* isa_last_error(void) { return g_last_error.c_str(); }
 const char* isa_version(void) { return "isa-b200 0.1 sm_100a"; }
 
 isa_status isa_set_wait_timeout_ns(uint64_t ns) {
-  g_timeout_ns = ns ? ns : kDefaultTimeoutNs;
+  g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs, std::memory_order_relaxed);
   return ISA_OK;
 }
 
 isa_status isa_set_fault_injection(int32_t mode) {
   if (mode != 0 && mode != 1) return fail(ISA_ERR_INVALID_ARG, "fault injection mode must be 0 or 1");
-  g_inject = mode;
+  g_inject.store(mode, std::memory_order_relaxed);
   return ISA_OK;
 }
 
