@@ -1,4 +1,4 @@
-"""Python binding of the ISA (In-context Sparse Attention) forward library.
+"""Python binding of the ISA (In-context Sparse Attention) library: forward and backward.
 
 Thin ctypes layer over ``libisa.so`` (entry points in include/isa.h): it
 marshals torch tensor pointers, sizes and the current CUDA stream and turns
