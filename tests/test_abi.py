@@ -56,6 +56,19 @@ def test_invalid_params_rejected_on_host(isa, bad, status):
     assert len(isa.load_library().isa_last_error()) > 0
 
 
+def test_block_limits(isa):
+    """8192 blocks and 6144 kept blocks per head are the largest plan
+    accepted; one block more of either is refused before anything runs."""
+    ok = isa.make_params(1, 1, 128, 131072, 131072, 32, 0.5)
+    v, _ = fake_view(isa, ok)
+    assert (v.T, v.T_kv) == (8192, 6144)
+    for bad in (isa.make_params(1, 1, 128, 131072, 131073, 32, 0.25),            # T = 8193
+                isa.make_params(1, 1, 128, 131072, 131072, 32, 2049 / 4096)):   # T_kv = 6145
+        with pytest.raises(isa.IsaError) as e:
+            isa.workspace_size(bad)
+        assert e.value.status == 2 and "at most" in str(e.value)
+
+
 def fake_view(isa, p):
     """Sizes from isa_plan_view_get; the workspace is never dereferenced."""
     lib = isa.load_library()
