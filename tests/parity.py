@@ -1,4 +1,5 @@
-"""Comparison helpers shared by the GPU parity tests (CPU-side logic only).
+"""Comparison helpers shared by the GPU parity tests, and the forward case
+runner (`check_case`) that several of them use.
 
 Index sets are compared with the margin rule of the ISA forward spec: an
 element may differ between the CUDA plan and the fp64 oracle only where its
@@ -16,7 +17,7 @@ import numpy as np
 import torch
 
 import oracle as O
-from workloads import Workload, bf16_to_f64
+from workloads import Workload, bf16_to_f64, generate_bits
 
 MARGIN_CTX = 1e-3
 MARGIN_EXACT = 1e-3
@@ -168,6 +169,63 @@ def head_inputs_f64(bits_q, bits_k, bits_v, h):
     return bf16_to_f64(bits_q[h]), bf16_to_f64(bits_k[h]), bf16_to_f64(bits_v[h])
 
 
+# ----------------------------------------------------------------------------
+# one forward case end to end: CUDA plan + forward, oracle, comparison
+# ----------------------------------------------------------------------------
+
+def params_of(isa, w: Workload):
+    return isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
+
+
+def run_isa(isa, w: Workload, bits=None):
+    qb, kb, vb = bits if bits is not None else generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    ws = isa.plan(q, k, v, p)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device="cuda")
+    out = isa.forward(q, k, v, ws, p, lse=lse)
+    torch.cuda.synchronize()
+    view = plan_view_host(isa.plan_view(p, ws))
+    return (qb, kb, vb), out.float().cpu().numpy().reshape(w.BH, w.L, w.D), \
+        lse.cpu().numpy().reshape(w.BH, w.L), view
+
+
+def check_case(isa, w: Workload, heads=None, blocks_per_head=None, max_moved_frac=0.02):
+    bits, out, lse, view = run_isa(isa, w)
+    assert int(view["status"][0]) == 0
+    qb, kb, vb = (x.reshape(w.BH, w.L, w.D) for x in bits)
+    p = oracle_params(w)
+    heads = range(w.BH) if heads is None else heads
+    n_blocks = n_moved = 0
+    worst = (0.0, 0.0)
+    for h in heads:
+        q, k, v = bf16_to_f64(qb[h]), bf16_to_f64(kb[h]), bf16_to_f64(vb[h])
+        pl = O.plan_head(q, k, v, p)
+        r = check_head_plan(pl, view, h)
+        assert not r.errors, (h, r.errors[:5])
+        if not r.ctx_equal:
+            n_moved += pl.T
+            n_blocks += pl.T
+            continue
+        blocks = list(range(pl.T))
+        if blocks_per_head is not None:
+            g = np.random.default_rng(1000 + h)
+            blocks = sorted(g.choice(pl.T, size=min(blocks_per_head, pl.T), replace=False).tolist())
+        moved = set(r.split_moved) | set(r.exact_moved)
+        use = [b for b in blocks if b not in moved]
+        n_blocks += len(blocks)
+        n_moved += len(blocks) - len(use)
+        ref, ref_lse = O.forward_head(q, k, v, pl, p, blocks=use)
+        rows = block_rows(pl, use)
+        mx, mean = compare_outputs(out[h], ref, rows)
+        worst = (max(worst[0], mx), max(worst[1], mean))
+        assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (h, mx, mean)
+        lerr = np.abs(lse[h][rows] - ref_lse[rows]).max() if len(rows) else 0.0
+        assert lerr <= 2e-2, (h, lerr)
+    assert n_moved <= max_moved_frac * max(n_blocks, 1), (n_moved, n_blocks)
+    return worst
+
+
 __all__ = ["topk_agrees", "check_head_plan", "compare_outputs", "block_rows", "plan_view_host", "oracle_params",
-           "to_torch_bf16", "head_inputs_f64", "energy_from_oracle", "MARGIN_CTX", "MARGIN_EXACT",
-           "MARGIN_SPLIT_REL", "OUT_MAX_ABS", "OUT_MEAN_ABS"]
+           "to_torch_bf16", "head_inputs_f64", "energy_from_oracle", "params_of", "run_isa", "check_case",
+           "MARGIN_CTX", "MARGIN_EXACT", "MARGIN_SPLIT_REL", "OUT_MAX_ABS", "OUT_MEAN_ABS"]

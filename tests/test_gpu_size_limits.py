@@ -9,7 +9,7 @@ outputs of a seeded sample of query blocks element by element."""
 import pytest
 import torch
 
-from test_gpu_parity import check_case
+from parity import check_case
 from workloads import Workload
 
 pytestmark = pytest.mark.gpu
