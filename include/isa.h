@@ -111,7 +111,7 @@ isa_status isa_plan_workspace_size(const isa_params* p, size_t* bytes);
  *   q, k, v : device, bf16 [B,H,L,D]
  *   ws      : device, at least isa_plan_workspace_size bytes, 256-byte
  *             aligned; overwritten; holds the plan afterwards
- * Launches 5 kernels on `stream`. */
+ * Launches 6 kernels on `stream` (5 when no block is flat). */
 isa_status isa_plan(const isa_params* p, const void* q, const void* k, const void* v,
                     void* ws, size_t ws_bytes, void* stream);
 
