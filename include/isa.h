@@ -192,8 +192,9 @@ isa_status isa_backward_workspace_size(const isa_params* p, size_t* bytes);
  *                 aligned; caller-owned scratch, rewritten by every call
  * P is recomputed from lse (no attention matrix is stored); products run in
  * bf16 on the tensor cores with fp32 accumulation, P and dS rounded to bf16.
- * Launches 5 kernels (4 when every kept block is exact for every flat
- * block, or no block is flat; one more when every context block is kept).
+ * Launches 5 kernels: one fewer when no flat block has a pooled column
+ * (every kept block exact, or no block flat), and one fewer when every
+ * context block is kept (no unkept tokens to zero).
  * Device timeouts go to the plan's status word, as for isa_forward. */
 isa_status isa_backward(const isa_params* p, const void* q, const void* k, const void* v, const void* ws,
                         size_t ws_bytes, const void* out, const float* lse, const void* dout, void* dq, void* dk,
