@@ -176,14 +176,15 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.out = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        self.out = os.fdopen(fd, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         # nvidia-smi takes a moment to start: wait (at most 3 s) for its first
@@ -205,6 +206,8 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.out is not None:
+            self.out.close()
 
     def summary(self):
         rows = []
