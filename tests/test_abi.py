@@ -56,6 +56,13 @@ def test_invalid_params_rejected_on_host(isa, bad, status):
     assert len(isa.load_library().isa_last_error()) > 0
 
 
+def test_binding_defaults_match_the_oracle(isa):
+    b = isa.make_params(1, 1, 64, 1, 1)
+    o = O.Params(D=64, L_src=1, L_ctx=1)
+    assert (b.alpha_s, b.alpha_f, b.alpha_ns, b.block) == (o.alpha_s, o.alpha_f, o.alpha_ns, o.block)
+    assert b.scale == 0.0 and o.scale is None       # both select 1/sqrt(D)
+
+
 def test_block_limits(isa):
     """8192 blocks and 6144 kept blocks per head are the largest plan
     accepted; one block more of either is refused before anything runs."""

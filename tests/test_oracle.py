@@ -187,6 +187,16 @@ def test_counts_follow_ratios():
     assert O.n_exact_blocks(0.0, 288) == 0 and O.n_exact_blocks(1.0, 288) == 288
 
 
+def test_default_ratios_are_the_pages_settings():
+    """The summary card's "Core method" section states the defaults as
+    sparsity rates: the context pre-selection removes 87.5 % of the context
+    blocks, half of the query blocks take the Taylor path, and the Taylor
+    path is 93.75 % sparse (the techwalker.com retelling, section 9, gives
+    alpha_ns = 0.0625); step (1) blocks 64 tokens."""
+    p = O.Params(D=64, L_src=1, L_ctx=1)
+    assert (1.0 - p.alpha_s, p.alpha_f, 1.0 - p.alpha_ns, p.block) == (0.875, 0.5, 0.9375, 64)
+
+
 def test_exact_share_counts_the_kept_blocks():
     """alpha_ns is a share of the KV blocks the flat path sees, the kept ones
     (techwalker.com retelling, section 9: alpha_ns = 0.0625 sends 6.25 % of
