@@ -43,6 +43,14 @@ second reading is plausible; the defaults are the ones the CUDA path uses):
     of S without a softmax (``sharp_cols="src"``, ``sharp_softmax=False``).
   * Ties: TopK keeps the lower index on equal scores; in the sharpness order
     the lower block index counts as sharper.
+  * alpha_f is the share of query blocks on the Taylor path ([R] step (3):
+    the top 1 - alpha_f by sharpness stay exact).  [R]'s Fig. 8 caption and
+    limitations paragraph and [T] section 9 describe a lower alpha_f as
+    sending more blocks to the approximation, the other direction; at the
+    default 0.5 both readings give the same split.
+  * A flat block's exact blocks are the kept blocks with the largest coarse
+    score in its row of S ([R] step (5) names no rule; [T] section 5 lets the
+    coarse relevance map decide).
   * alpha_ns counts blocks of the kept KV (``ns_base="kept"``), following [T]
     section 9 (6.25% of KV blocks exact, 93.75% approximated); [R] step (5)
     says "total block count" (``ns_base="all"``: ceil(alpha_ns * T)).
