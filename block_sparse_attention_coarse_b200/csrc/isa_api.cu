@@ -151,7 +151,6 @@ void init_once() {
   g_init_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
   if (g_init_err == cudaSuccess && q != cudaDriverEntryPointSuccess) g_init_err = cudaErrorNotSupported;
   g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-  if (g_init_err == cudaSuccess) g_init_err = prepare_plan_kernels();
 }
 
 isa_status ensure_init() {

@@ -77,7 +77,6 @@ struct BwdArgs {
 // launchers (host)
 cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
                         cudaStream_t st);
-cudaError_t prepare_plan_kernels();
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_backward(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sm_count, cudaStream_t st);
 size_t coarse_backward_bytes(const Dims& d);

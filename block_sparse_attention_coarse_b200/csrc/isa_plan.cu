@@ -410,8 +410,9 @@ static cudaError_t launch_plan_d(const Dims& dm, const void* q, const void* k, c
   return cudaSuccess;
 }
 
-cudaError_t prepare_plan_kernels() {
-  // several planning kernels need more than the default 48 KB of dynamic shared memory
+// Several planning kernels need more than the default 48 KB of dynamic
+// shared memory; the limit is raised on each device before its first plan.
+static cudaError_t prepare_plan_kernels() {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(rowstats_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)rowstats_smem(64))) != cudaSuccess) return e;
@@ -431,6 +432,9 @@ cudaError_t prepare_plan_kernels() {
 
 cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
                         cudaStream_t st) {
+  static std::atomic<unsigned long long> attr_done{0};
+  const cudaError_t e = once_per_device(attr_done, prepare_plan_kernels);
+  if (e != cudaSuccess) return e;
   return dm.D == 64 ? launch_plan_d<64>(dm, q, k, v, pp, st) : launch_plan_d<128>(dm, q, k, v, pp, st);
 }
 
