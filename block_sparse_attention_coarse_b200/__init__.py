@@ -39,7 +39,7 @@ ISA_ERR_DEVICE_TIMEOUT = 5
 EXPORTS = (
     "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
-    "isa_forward_static", "isa_rope_workspace_size", "isa_rope", "isa_backward_workspace_size", "isa_backward",
+    "isa_forward_static", "isa_forward_static_status", "isa_rope_workspace_size", "isa_rope", "isa_backward_workspace_size", "isa_backward",
     "isa_coarse_residual", "isa_coarse_residual_backward_workspace_size", "isa_coarse_residual_backward",
 )
 
@@ -95,6 +95,8 @@ def load_library() -> ctypes.CDLL:
     lib.isa_set_fault_injection.argtypes = [ctypes.c_int32]
     lib.isa_forward_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.isa_forward_static.restype = ctypes.c_int
+    lib.isa_forward_static_status.argtypes = [ctypes.c_int32, vp, vp]
+    lib.isa_forward_static_status.restype = ctypes.c_int
     lib.isa_rope_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.isa_rope.argtypes = [P, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]
     lib.isa_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
@@ -417,28 +419,3 @@ def set_wait_timeout_ns(ns: int) -> None:
 
 def set_fault_injection(mode: int) -> None:
     _check(load_library().isa_set_fault_injection(int(mode)))
-
-
-def executed_flops(p: Params, view: Dict[str, object]) -> float:
-    """Algorithmic work of one ISA forward from a plan view copied to the
-    host: 4*D per (query token, key column) pair -- an exact key token is one
-    column, a pooled block one column -- plus 2*T*T*D per head for the
-    coarse scores."""
-    import numpy as np
-    b = p.block
-    T_src, T = int(view["T_src"]), int(view["T"])
-    cnt = np.array([min(b, p.L_src - j * b) for j in range(T_src)] +
-                   [min(b, p.L_ctx - c * b) for c in range(T - T_src)], np.float64)
-    kept = view["kept"].cpu().numpy()
-    sharp = view["sharp_ids"].cpu().numpy()
-    flat = view["flat_ids"].cpu().numpy()
-    exact = view["exact"].cpu().numpy()
-    T_kv, n_ex = int(view["T_kv"]), int(view["n_exact"])
-    total = 0.0
-    for h in range(kept.shape[0]):
-        kv_tokens = cnt[kept[h]].sum()
-        total += cnt[sharp[h]].sum() * kv_tokens
-        if flat.shape[1]:
-            ex_tok = cnt[kept[h][exact[h]]].sum(axis=1) if n_ex else np.zeros(flat.shape[1])
-            total += float((cnt[flat[h]] * (ex_tok + (T_kv - n_ex))).sum())
-    return 4.0 * p.D * total + 2.0 * T * T * p.D * kept.shape[0]

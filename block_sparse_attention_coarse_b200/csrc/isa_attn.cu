@@ -297,13 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (I.kind == 0) {
         jm1 = (a.L - 1) / 128;
       }
-      int ekk[G];
-      load_exact<G>(a, I, 0, ekk);
+      int ekk = load_exact(a, I, 0, g_r);
       for (int j = 0; j < I.ntiles; ++j, ++t) {
         TileMeta cur;
         if (I.kind == 2 || j == jm0 || j == jm1) {
           cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
-          load_exact<G>(a, I, j + 1, ekk);
+          ekk = load_exact(a, I, j + 1, g_r);
         } else {
           cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
           cur.pooled = 0;
@@ -316,9 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t sr[2][32];
-        tmem_ld16x2_32<64>(trow + buf * 128, sr[0]);        // columns 64h + 0..31
-        tmem_ld16x2_32<64>(trow + buf * 128 + 32, sr[1]);   // columns 64h + 32..63
-        tmem_wait_ld();
+        // columns 64h + 0..31 and 64h + 32..63, waited for in the same statement
+        tmem_ld16x2_sync2<64>(trow + buf * 128, sr[0], trow + buf * 128 + 32, sr[1]);
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
@@ -396,8 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 32) {
             uint32_t o[32];
-            tmem_ld16x2_32<DH>(trow + kTmemO + c0, o);   // columns DH*h + c0..+31
-            tmem_wait_ld();
+            tmem_ld16x2_sync1<DH>(trow + kTmemO + c0, o);   // columns DH*h + c0..+31
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st16x2_32<DH>(trow + kTmemO + c0, o);
@@ -417,9 +414,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_ready, n & 1, wc))) break;
       tc_fence_after();
       uint32_t o[DH / 32][32];
-#pragma unroll
-      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld16x2_32<DH>(trow + kTmemO + 32 * c0, o[c0]);
-      tmem_wait_ld();
+      if constexpr (DH == 64) {
+        tmem_ld16x2_sync2<DH>(trow + kTmemO, o[0], trow + kTmemO + 32, o[DH / 64]);
+      } else {
+        tmem_ld16x2_sync1<DH>(trow + kTmemO, o[0]);
+      }
       tc_fence_before();
       mbar_arrive(&o_free);
       const float l_tot = l_run + __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);

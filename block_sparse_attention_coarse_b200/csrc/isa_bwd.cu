@@ -504,16 +504,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc_fence_after();
         const int last = meta[s].last;
         const bool on = row_valid && ((meta[s].m[gq][r >> 5] >> (r & 31)) & 1u);
-        uint32_t sv[16], dp[16];
-        tmem_ld16(tl + kTST + buf * 64 + 16 * qd, sv);
-        tmem_ld16(tl + kTDP + buf * 64 + 16 * qd, dp);
         // (lse2, Delta) of this thread's 16 columns, two columns per 16-byte
         // broadcast load; rows past a block's end hold (inf, 0), so P = 0 there
         const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE) + (gq * R + coff) / 2;
         float4 ld[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) ld[e] = dls[e];
-        tmem_wait_ld();
+        uint32_t sv[16], dp[16];
+        tmem_ld16_pair_sync(tl + kTST + buf * 64 + 16 * qd, sv, tl + kTDP + buf * 64 + 16 * qd, dp);
         uint32_t pp[8], pd[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
@@ -538,59 +536,53 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       // epilogue: this thread's DQ columns of dV and dK for tile row r
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_ready, n & 1, wc))) break;
       tc_fence_after();
-      uint32_t gv[DQ / 16][16], gk[DQ / 16][16];
-#pragma unroll
-      for (int c0 = 0; c0 < DQ / 16; ++c0) {
-        tmem_ld16(tl + kTDV + qd * DQ + 16 * c0, gv[c0]);
-        tmem_ld16(tl + kTDV + D + qd * DQ + 16 * c0, gk[c0]);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&acc_free);
-      if (!row_valid) continue;
+      // dV first, then dK, so that only one of them is held in registers
       const float sc = b.scale;
-      if (pooled) {
-        float4* kd = reinterpret_cast<float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
-        float4* vd = reinterpret_cast<float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
+      const float inv = 1.f / (float)nj;
 #pragma unroll
-        for (int e = 0; e < DQ; e += 4) {
-          const uint32_t* k4 = &gk[e >> 4][e & 15];
-          const uint32_t* v4 = &gv[e >> 4][e & 15];
-          kd[e >> 2] = make_float4(sc * __uint_as_float(k4[0]), sc * __uint_as_float(k4[1]),
-                                   sc * __uint_as_float(k4[2]), sc * __uint_as_float(k4[3]));
-          vd[e >> 2] = make_float4(__uint_as_float(v4[0]), __uint_as_float(v4[1]), __uint_as_float(v4[2]),
-                                   __uint_as_float(v4[3]));
+      for (int part = 0; part < 2; ++part) {   // 0: dV, 1: dK (scaled by s)
+        uint32_t g[DQ / 16][16];
+        const uint32_t col = kTDV + part * D + qd * DQ;
+        __syncwarp();
+        if constexpr (DQ == 32) {
+          tmem_ld16_pair_sync(tl + col, g[0], tl + col + 16, g[DQ / 32]);
+        } else {
+          tmem_ld16_sync(tl + col, g[0]);
         }
-      } else {
-        // this block's share of its pooled-mean gradient: dKc_j / n_j, dVc_j / n_j
-        const float inv = 1.f / (float)nj;
-        const float4* kc = reinterpret_cast<const float4*>(b.dKc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
-        const float4* vc = reinterpret_cast<const float4*>(b.dVc + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
-        uint4* kd = reinterpret_cast<uint4*>(b.dk + ((size_t)bh * a.L + tok) * D + qd * DQ);
-        uint4* vd = reinterpret_cast<uint4*>(b.dv + ((size_t)bh * a.L + tok) * D + qd * DQ);
+        if (part == 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_free);
+        }
+        if (!row_valid) continue;
+        const float f = part ? sc : 1.f;
+        if (pooled) {
+          float4* dst = reinterpret_cast<float4*>((part ? b.dKc : b.dVc) + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
 #pragma unroll
-        for (int e = 0; e < DQ; e += 8) {
-          float xk[8], xv[8];
+          for (int e = 0; e < DQ; e += 4) {
+            const uint32_t* g4 = &g[e >> 4][e & 15];
+            dst[e >> 2] = make_float4(f * __uint_as_float(g4[0]), f * __uint_as_float(g4[1]),
+                                      f * __uint_as_float(g4[2]), f * __uint_as_float(g4[3]));
+          }
+        } else {
+          // this block's share of its pooled-mean gradient: dKc_j / n_j, dVc_j / n_j
+          const float4* pc =
+              reinterpret_cast<const float4*>((part ? b.dKc : b.dVc) + ((size_t)bh * a.T_kv_pad + kk) * D + qd * DQ);
+          uint4* dst = reinterpret_cast<uint4*>((part ? b.dk : b.dv) + ((size_t)bh * a.L + tok) * D + qd * DQ);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            xk[i] = sc * __uint_as_float(gk[(e + i) >> 4][(e + i) & 15]);
-            xv[i] = __uint_as_float(gv[(e + i) >> 4][(e + i) & 15]);
+          for (int e = 0; e < DQ; e += 8) {
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = f * __uint_as_float(g[(e + i) >> 4][(e + i) & 15]);
+            if (b.has_pooled) {
+              const float4 c0 = pc[e >> 2], c1 = pc[(e >> 2) + 1];
+              x[0] = fmaf(c0.x, inv, x[0]); x[1] = fmaf(c0.y, inv, x[1]);
+              x[2] = fmaf(c0.z, inv, x[2]); x[3] = fmaf(c0.w, inv, x[3]);
+              x[4] = fmaf(c1.x, inv, x[4]); x[5] = fmaf(c1.y, inv, x[5]);
+              x[6] = fmaf(c1.z, inv, x[6]); x[7] = fmaf(c1.w, inv, x[7]);
+            }
+            dst[e >> 3] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                     pack_bf16x2(x[6], x[7]));
           }
-          if (b.has_pooled) {
-            const float4 k0 = kc[e >> 2], k1 = kc[(e >> 2) + 1], v0 = vc[e >> 2], v1 = vc[(e >> 2) + 1];
-            xk[0] = fmaf(k0.x, inv, xk[0]); xk[1] = fmaf(k0.y, inv, xk[1]);
-            xk[2] = fmaf(k0.z, inv, xk[2]); xk[3] = fmaf(k0.w, inv, xk[3]);
-            xk[4] = fmaf(k1.x, inv, xk[4]); xk[5] = fmaf(k1.y, inv, xk[5]);
-            xk[6] = fmaf(k1.z, inv, xk[6]); xk[7] = fmaf(k1.w, inv, xk[7]);
-            xv[0] = fmaf(v0.x, inv, xv[0]); xv[1] = fmaf(v0.y, inv, xv[1]);
-            xv[2] = fmaf(v0.z, inv, xv[2]); xv[3] = fmaf(v0.w, inv, xv[3]);
-            xv[4] = fmaf(v1.x, inv, xv[4]); xv[5] = fmaf(v1.y, inv, xv[5]);
-            xv[6] = fmaf(v1.z, inv, xv[6]); xv[7] = fmaf(v1.w, inv, xv[7]);
-          }
-          kd[e >> 3] = make_uint4(pack_bf16x2(xk[0], xk[1]), pack_bf16x2(xk[2], xk[3]), pack_bf16x2(xk[4], xk[5]),
-                                  pack_bf16x2(xk[6], xk[7]));
-          vd[e >> 3] = make_uint4(pack_bf16x2(xv[0], xv[1]), pack_bf16x2(xv[2], xv[3]), pack_bf16x2(xv[4], xv[5]),
-                                  pack_bf16x2(xv[6], xv[7]));
         }
       }
     }
@@ -863,13 +855,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (ic.src_tail != a.b) jm0 = (a.T_src - 1) / G;
         jm1 = (a.T_kv - 1) / G;
       }
-      int ekk[G];
-      load_exact<G>(a, I, 0, ekk);
+      int ekk = load_exact(a, I, 0, g_r);
       for (int j = 0; j < I.ntiles; ++j, ++t) {
         TileMeta cur;
         if (I.kind == 2 || j == jm0 || j == jm1) {
           cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
-          load_exact<G>(a, I, j + 1, ekk);
+          ekk = load_exact(a, I, j + 1, g_r);
         } else {
           cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
           cur.pooled = 0;
@@ -881,35 +872,38 @@ __global__ void __launch_bounds__(kQThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[2][32], dr[2][32];
-        tmem_ld16x2_32<64>(trow + kTS + buf * 128, sr[0]);
-        tmem_ld16x2_32<64>(trow + kTS + buf * 128 + 32, sr[1]);
-        tmem_ld16x2_32<64>(trow + kTP, dr[0]);
-        tmem_ld16x2_32<64>(trow + kTP + 32, dr[1]);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&dp_free);   // dP of the next tile may overwrite the buffer
-        float s[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-        if (cur.masked) {
-          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = ((((c < 32) ? w0 : w1) >> (c & 31)) & 1u) ? s[c] : -INFINITY;
-          if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
-            const int kk0 = (j - a.n_exact) * 128 + 64 * h;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
-          }
-        }
+        // S and dP, 32 columns of this thread's half row at a time (64
+        // registers per round instead of 128)
         const float neg = (cur.pooled ? log2b : 0.f) - mine.x;
+        const uint32_t wsel[2] = {h ? cur.mw[2] : cur.mw[0], h ? cur.mw[3] : cur.mw[1]};
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2(fmaf(s[c], sl2, neg)), p1 = ex2(fmaf(s[c + 1], sl2, neg));
-          const float g0 = p0 * (__uint_as_float(dr[c >> 5][c & 31]) - mine.y);
-          const float g1 = p1 * (__uint_as_float(dr[(c + 1) >> 5][(c + 1) & 31]) - mine.y);
-          pk[c >> 1] = pack_bf16x2(g0, g1);
+        for (int part = 0; part < 2; ++part) {
+          uint32_t sr[32], dr[32];
+          tmem_ld16x2_sync2<64>(trow + kTS + buf * 128 + 32 * part, sr, trow + kTP + 32 * part, dr);
+          if (part == 1) {
+            tc_fence_before();
+            mbar_arrive(&dp_free);   // dP of the next tile may overwrite the buffer
+          }
+          float s[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(sr[c]);
+          if (cur.masked) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) s[c] = ((wsel[part] >> c) & 1u) ? s[c] : -INFINITY;
+            if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
+              const int kk0 = (j - a.n_exact) * 128 + 64 * h + 32 * part;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2(fmaf(s[c], sl2, neg)), p1 = ex2(fmaf(s[c + 1], sl2, neg));
+            const float g0 = p0 * (__uint_as_float(dr[c]) - mine.y);
+            const float g1 = p1 * (__uint_as_float(dr[c + 1]) - mine.y);
+            pk[16 * part + (c >> 1)] = pack_bf16x2(g0, g1);
+          }
         }
         tmem_st16x2_32<32>(trow + kTS + buf * 128, pk);   // dS keys 64h..64h+63 -> columns 32h..32h+31
         tmem_wait_st();
@@ -921,9 +915,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&dq_ready, n & 1, wc))) break;
       tc_fence_after();
       uint32_t o[DH / 32][32];
-#pragma unroll
-      for (int c0 = 0; c0 < DH / 32; ++c0) tmem_ld16x2_32<DH>(trow + kTQ + 32 * c0, o[c0]);
-      tmem_wait_ld();
+      if constexpr (DH == 64) {
+        tmem_ld16x2_sync2<DH>(trow + kTQ, o[0], trow + kTQ + 32, o[DH / 64]);
+      } else {
+        tmem_ld16x2_sync1<DH>(trow + kTQ, o[0]);
+      }
       tc_fence_before();
       mbar_arrive(&dq_free);
       if (row_valid) {

@@ -108,21 +108,17 @@ struct TileMeta {
   int pooled, masked;
 };
 
-// exact-block positions (in the kept list) of the G query blocks of a flat
-// item for exact tile j: loaded one tile ahead of their use
-template <int G>
-__device__ __forceinline__ void load_exact(const AttnArgs& a, const Item& I, int j, int (&kk)[G]) {
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const int f = I.slot0 + g;
-    kk[g] = (I.kind == 2 && j < a.n_exact && f < a.n_flat) ? a.exact[((size_t)I.bh * a.n_flat + f) * a.n_exact + j]
-                                                             : -1;
-  }
+// exact-block position (in the kept list) of query block g_r of a flat item
+// for exact tile j (-1 outside the exact tiles): loaded one tile ahead of its
+// use; a row needs only its own query block's entry
+__device__ __forceinline__ int load_exact(const AttnArgs& a, const Item& I, int j, int g_r) {
+  const int f = I.slot0 + g_r;
+  return (I.kind == 2 && j < a.n_exact && f < a.n_flat) ? a.exact[((size_t)I.bh * a.n_flat + f) * a.n_exact + j] : -1;
 }
 
 template <int R, int G>
 __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, const ItemCounts& ic, int j, int g_r,
-                                              const uint32_t* rbits, const int (&ekk)[G]) {
+                                              const uint32_t* rbits, int ekk_r) {
   TileMeta m;
   if (I.kind == 2 && j >= a.n_exact) {
     // pooled tile: kept blocks [jp*128, jp*128+128) minus this row's exact blocks
@@ -148,7 +144,7 @@ __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, 
     } else if (I.kind == 1) {
       cnt[g] = kept_count(a, ic, j * G + g);
     } else {
-      cnt[g] = (g == g_r) ? kept_count(a, ic, ekk[g]) : 0;   // block-diagonal exact tiles
+      cnt[g] = (g == g_r) ? kept_count(a, ic, ekk_r) : 0;   // block-diagonal exact tiles
     }
   }
   bool full = true;
@@ -163,17 +159,53 @@ __device__ __forceinline__ TileMeta tile_meta(const AttnArgs& a, const Item& I, 
   return m;
 }
 
-// TMEM access of 16 lanes with the columns split between the two half warps
+// TMEM loads of 16 lanes with the columns split between the two half warps
 // (the .16x32bx2 shape): thread t < 16 reaches lane base+t, columns
 // [c, c+32); thread t >= 16 reaches lane base+t-16, columns [c+SPLIT,
-// c+SPLIT+32).  So both 64-column halves of a row sit in one warp.
+// c+SPLIT+32).  So both 64-column halves of a row sit in one warp.  Each
+// helper issues its groups and their tcgen05.wait::ld in one asm statement
+// (see tmem_ld16_pair_sync).  One group:
 template <int SPLIT>
-__device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld16x2_sync1(uint32_t t0, uint32_t (&r0)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
-      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
-      : ISA_R32(r)
-      : "r"(taddr), "n"(SPLIT));
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ISA_R32(r0)
+      : "r"(t0), "n"(SPLIT)
+      : "memory");
+}
+// Two groups and the wait:
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld16x2_sync2(uint32_t t0, uint32_t (&r0)[32], uint32_t t1, uint32_t (&r1)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64], %66;\n\t"
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65], %66;\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ISA_R32(r0), ISA_R32(r1)
+      : "r"(t0), "r"(t1), "n"(SPLIT)
+      : "memory");
+}
+// Four groups and the wait:
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld16x2_sync4(uint32_t t0, uint32_t (&r0)[32], uint32_t t1, uint32_t (&r1)[32],
+                                                  uint32_t t2, uint32_t (&r2)[32], uint32_t t3, uint32_t (&r3)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128], %132;\n\t"
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129], %132;\n\t"
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130], %132;\n\t"
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,"
+      "%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131],"
+      " %132;\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ISA_R32(r0), ISA_R32(r1), ISA_R32(r2), ISA_R32(r3)
+      : "r"(t0), "r"(t1), "r"(t2), "r"(t3), "n"(SPLIT)
+      : "memory");
 }
 template <int SPLIT>
 __device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const uint32_t (&r)[32]) {

@@ -154,15 +154,29 @@ isa_status isa_dense(const isa_params* p, const void* q, const void* k, const vo
  *  - A problem whose plan needs more than 16 MiB (isa_plan_workspace_size)
  *    returns ISA_ERR_WORKSPACE with a message; nothing is launched.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
- *  - Allocates nothing (no cudaMalloc/cudaFree, no library allocation).
+ *    (cudaGetSymbolAddress), which may make the driver load the library's
+ *    device code and the array with it: make that first call, per device,
+ *    as a warm-up where allocation is allowed, and before any stream capture.
+ *    Later calls allocate nothing (no cudaMalloc/cudaFree, no library
+ *    allocation).
+ *  - The looked-up address is cached per device; after cudaDeviceReset it is
+ *    stale, so do not call this entry point on that device again.
  *  - All calls share the one array, which keeps the last call's contents;
  *    every plan entry is rewritten and the status word cleared by each call.
  *    Calls that overlap on the GPU race on the array: order them.
- * Device timeouts are reported as for isa_forward, in the array's status
- * word (not readable by the caller; use isa_plan/isa_forward to inspect). */
+ * Device timeouts are written to the array's status word; read it with
+ * isa_forward_static_status. */
 isa_status isa_forward_static(const isa_params* p, const void* q, const void* k, const void* v, void* out,
                               float* lse, void* stream);
+
+/* Copies the status word of isa_forward_static's array on CUDA device
+ * `device` (ISA_OK, or ISA_ERR_DEVICE_TIMEOUT after a device wait ran out)
+ * to `dst` (4 bytes of host or device memory) with one stream-ordered copy
+ * on `stream`: the value is there once the stream has reached the copy (for
+ * pageable host memory, when the call returns).  Like the entry point it
+ * serves, it has no counterpart on the pages.  Returns ISA_ERR_INVALID_ARG
+ * when dst is NULL or isa_forward_static has not run on that device. */
+isa_status isa_forward_static_status(int32_t device, int32_t* dst, void* stream);
 
 /* Workspace of isa_backward: (lse * log2 e, rowsum(dout * out)) for every
  * row of every block, padded to `block` rows per block (B*H * T * block * 8

@@ -8,10 +8,19 @@ set, in that set's own units:
   context TopK       : absolute 1e-3 on imp / T_src (the mean coarse score)
   flat exact TopK    : absolute 1e-3 on S
   sharp/flat split   : relative 1e-3 on E_i = sum_j softmax(S_i)_j^2
+
+Where a CUDA index set differs from the oracle's only inside the margin,
+both are valid plans of the method (the choice between near-equal scores is
+not unique).  The output check then runs the oracle on the CUDA plan's
+index sets (`plan_from_gpu`), after each set has passed the margin rule
+against the oracle's own fp64 scores; every value the oracle uses (pooled
+means, coarse scores, inputs) stays its own.  So no block and no head is
+left out of the output comparison.
 """
 from __future__ import annotations
 
-from typing import Iterable, List, Sequence, Tuple
+import dataclasses
+from typing import Iterable, List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -66,20 +75,30 @@ class HeadCheck:
     def __init__(self):
         self.ctx_equal = True
         self.split_moved: List[int] = []      # blocks whose sharp/flat side differs
-        self.exact_moved: List[int] = []      # flat blocks whose exact list differs
+        self.exact_moved: List[int] = []      # flat blocks whose exact list differs from the oracle's
         self.errors: List[str] = []
         self.outside_margin: List[str] = []   # set differences beyond the margins (inputs_equal=False)
+
+
+def gpu_kept(pl: O.HeadPlan, gpu: dict, h: int) -> np.ndarray:
+    """The kept block ids implied by the CUDA plan's context selection."""
+    return np.concatenate([np.arange(pl.T_src), pl.T_src + np.sort(gpu["ctx_sel"][h])]).astype(np.int64)
 
 
 def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int, inputs_equal: bool = True) -> HeadCheck:
     """Compares plan arrays of head `h` (host numpy copies of the plan view)
     with the oracle plan `pl` under the margin rules.
 
+    The exact list of every CUDA flat block is checked against the oracle's
+    coarse scores over the CUDA plan's own kept set (the same set as the
+    oracle's when the context selections agree), so a within-margin context
+    or split difference does not hide the exact lists from the check.
+
     inputs_equal=False: the two sides planned from inputs that may differ by
     one bf16 rounding per element (each side applied its own position
     embedding): value tolerances widen to cover that, and index-set
-    differences beyond the margins are recorded in `outside_margin` (to be
-    counted as moved blocks) instead of failing."""
+    differences beyond the margins are recorded in `outside_margin` instead
+    of failing."""
     r = HeadCheck()
     T_src = pl.T_src
     tol_pool, tol_imp, tol_energy = (1e-5, 1e-3, 1e-4) if inputs_equal else (2.0 ** -8, 2e-2, 2e-2)
@@ -99,8 +118,8 @@ def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int, inputs_equal: bool = True
     if list(gpu["ctx_sel"][h]) != sorted(gpu["ctx_sel"][h]):
         r.errors.append("ctx_sel not ascending")
     r.ctx_equal = np.array_equal(np.sort(gpu["ctx_sel"][h]), pl.ctx_sel)
-    kept_gpu = gpu["kept"][h]
-    if not np.array_equal(kept_gpu, np.concatenate([np.arange(T_src), T_src + np.sort(gpu["ctx_sel"][h])])):
+    kept = gpu_kept(pl, gpu, h)
+    if not np.array_equal(gpu["kept"][h], kept):
         r.errors.append("kept list inconsistent with ctx_sel")
     # energy and split
     E = energy_from_oracle(pl)
@@ -120,25 +139,41 @@ def check_head_plan(pl: O.HeadPlan, gpu: dict, h: int, inputs_equal: bool = True
         if not ok:
             margin_fail.append("sharp set outside margin")
     r.split_moved = sorted(set(sharp_gpu.tolist()).symmetric_difference(pl.sharp.tolist()))
-    # exact lists, where the kept sets agree
-    if r.ctx_equal:
-        flat_pos_gpu = {int(b): i for i, b in enumerate(flat_gpu)}
-        for ro, b in enumerate(pl.flat):
-            if int(b) not in flat_pos_gpu:
-                continue
-            got = gpu["exact"][h][flat_pos_gpu[int(b)]]
-            ok, diff = topk_agrees(pl.S[b, pl.kept], pl.exact.shape[1], got, MARGIN_EXACT)
-            if not ok:
-                margin_fail.append(f"exact list of block {b} outside margin")
-            if list(got) != sorted(got):
-                r.errors.append("exact list not ascending")
-            bits = gpu["exact_bits"][h][flat_pos_gpu[int(b)]].astype(np.uint32)
-            from_bits = [i for i in range(len(pl.kept)) if (bits[i // 32] >> (i % 32)) & 1]
-            if from_bits != sorted(got.tolist()):
-                r.errors.append(f"exact bitmap of block {b} disagrees with the list")
-            if diff:
-                r.exact_moved.append(int(b))
+    # exact lists of every CUDA flat block, over the CUDA plan's kept set
+    n_ex = pl.exact.shape[1]
+    flat_pos_oracle = {int(b): i for i, b in enumerate(pl.flat)}
+    for ro, b in enumerate(flat_gpu):
+        b = int(b)
+        got = gpu["exact"][h][ro]
+        ok, diff = topk_agrees(pl.S[b, kept], n_ex, got, MARGIN_EXACT)
+        if not ok:
+            margin_fail.append(f"exact list of block {b} outside margin")
+        if list(got) != sorted(got):
+            r.errors.append("exact list not ascending")
+        bits = gpu["exact_bits"][h][ro].astype(np.uint32)
+        from_bits = [i for i in range(len(kept)) if (bits[i // 32] >> (i % 32)) & 1]
+        if from_bits != sorted(got.tolist()):
+            r.errors.append(f"exact bitmap of block {b} disagrees with the list")
+        same_as_oracle = r.ctx_equal and b in flat_pos_oracle and \
+            np.array_equal(np.sort(got), pl.exact[flat_pos_oracle[b]])
+        if not same_as_oracle and n_ex:
+            r.exact_moved.append(b)
     return r
+
+
+def plan_from_gpu(pl: O.HeadPlan, gpu: dict, h: int) -> O.HeadPlan:
+    """The oracle's plan of head h with the CUDA plan's index sets (kept
+    context blocks, sharp/flat split, exact lists) in place of its own.
+
+    Only for a head whose CUDA sets `check_head_plan` accepted: each is then
+    a valid choice of the method under the margin rule (it differs from the
+    oracle's only between scores closer than the margin).  Pooled means,
+    coarse scores and token counts stay the oracle's fp64 values."""
+    kept = gpu_kept(pl, gpu, h)
+    flat = np.asarray(gpu["flat_ids"][h], np.int64)
+    exact = np.sort(np.asarray(gpu["exact"][h], np.int64).reshape(len(flat), -1), axis=1)
+    return dataclasses.replace(pl, ctx_sel=np.sort(np.asarray(gpu["ctx_sel"][h], np.int64)), kept=kept,
+                               sharp=np.asarray(gpu["sharp_ids"][h], np.int64), flat=flat, exact=exact)
 
 
 def compare_outputs(out_gpu: np.ndarray, out_ref: np.ndarray, rows: np.ndarray):
@@ -178,6 +213,10 @@ def params_of(isa, w: Workload):
 
 
 def run_isa(isa, w: Workload, bits=None):
+    """plan + forward on the GPU.  Returns the input bits, the output [BH, L, D]
+    and lse [BH, L] as device tensors (copied to the host head by head by the
+    caller: at 131072 tokens the whole output is 2.7 GB in fp32), and host
+    copies of the plan arrays."""
     qb, kb, vb = bits if bits is not None else generate_bits(w)
     q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
     p = params_of(isa, w)
@@ -186,11 +225,21 @@ def run_isa(isa, w: Workload, bits=None):
     out = isa.forward(q, k, v, ws, p, lse=lse)
     torch.cuda.synchronize()
     view = plan_view_host(isa.plan_view(p, ws))
-    return (qb, kb, vb), out.float().cpu().numpy().reshape(w.BH, w.L, w.D), \
-        lse.cpu().numpy().reshape(w.BH, w.L), view
+    del q, k, v, ws
+    return (qb, kb, vb), out.view(w.BH, w.L, w.D), lse.view(w.BH, w.L), view
 
 
-def check_case(isa, w: Workload, heads=None, blocks_per_head=None, max_moved_frac=0.02):
+def head_out(out: torch.Tensor, lse: torch.Tensor, h: int):
+    """Host float copies of one head's output rows and lse."""
+    return out[h].float().cpu().numpy(), lse[h].cpu().numpy()
+
+
+def check_case(isa, w: Workload, heads=None, blocks_per_head=None):
+    """Runs plan + forward on the GPU and compares, per checked head:
+    the plan under the margin rules, then the output and lse of every query
+    block (or a seeded sample of `blocks_per_head`) with the oracle run on
+    the GPU's validated plan.  Returns (worst max-abs, worst mean-abs,
+    blocks compared, blocks whose plan decision differs inside the margin)."""
     bits, out, lse, view = run_isa(isa, w)
     assert int(view["status"][0]) == 0
     qb, kb, vb = (x.reshape(w.BH, w.L, w.D) for x in bits)
@@ -203,29 +252,26 @@ def check_case(isa, w: Workload, heads=None, blocks_per_head=None, max_moved_fra
         pl = O.plan_head(q, k, v, p)
         r = check_head_plan(pl, view, h)
         assert not r.errors, (h, r.errors[:5])
-        if not r.ctx_equal:
-            n_moved += pl.T
-            n_blocks += pl.T
-            continue
         blocks = list(range(pl.T))
         if blocks_per_head is not None:
             g = np.random.default_rng(1000 + h)
             blocks = sorted(g.choice(pl.T, size=min(blocks_per_head, pl.T), replace=False).tolist())
-        moved = set(r.split_moved) | set(r.exact_moved)
-        use = [b for b in blocks if b not in moved]
+        moved = set(range(pl.T)) if not r.ctx_equal else set(r.split_moved) | set(r.exact_moved)
         n_blocks += len(blocks)
-        n_moved += len(blocks) - len(use)
-        ref, ref_lse = O.forward_head(q, k, v, pl, p, blocks=use)
-        rows = block_rows(pl, use)
-        mx, mean = compare_outputs(out[h], ref, rows)
+        n_moved += sum(1 for b in blocks if b in moved)
+        ref_plan = plan_from_gpu(pl, view, h)
+        ref, ref_lse = O.forward_head(q, k, v, ref_plan, p, blocks=blocks)
+        rows = block_rows(pl, blocks)
+        out_h, lse_h = head_out(out, lse, h)
+        mx, mean = compare_outputs(out_h, ref, rows)
         worst = (max(worst[0], mx), max(worst[1], mean))
         assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (h, mx, mean)
-        lerr = np.abs(lse[h][rows] - ref_lse[rows]).max() if len(rows) else 0.0
+        lerr = np.abs(lse_h[rows] - ref_lse[rows]).max() if len(rows) else 0.0
         assert lerr <= 2e-2, (h, lerr)
-    assert n_moved <= max_moved_frac * max(n_blocks, 1), (n_moved, n_blocks)
-    return worst
+    return worst[0], worst[1], n_blocks, n_moved
 
 
-__all__ = ["topk_agrees", "check_head_plan", "compare_outputs", "block_rows", "plan_view_host", "oracle_params",
-           "to_torch_bf16", "head_inputs_f64", "energy_from_oracle", "params_of", "run_isa", "check_case",
-           "MARGIN_CTX", "MARGIN_EXACT", "MARGIN_SPLIT_REL", "OUT_MAX_ABS", "OUT_MEAN_ABS"]
+__all__ = ["topk_agrees", "check_head_plan", "plan_from_gpu", "gpu_kept", "compare_outputs", "block_rows",
+           "plan_view_host", "oracle_params", "to_torch_bf16", "head_inputs_f64", "energy_from_oracle", "params_of",
+           "run_isa", "head_out", "check_case", "MARGIN_CTX", "MARGIN_EXACT", "MARGIN_SPLIT_REL", "OUT_MAX_ABS",
+           "OUT_MEAN_ABS"]

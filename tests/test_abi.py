@@ -205,3 +205,16 @@ def test_coarse_residual_arguments_rejected_before_launch(isa):
     assert b"dout is NULL" in lib.isa_last_error()
     assert lib.isa_coarse_residual_backward(*(args[:10] + [nc.value - 1] + args[11:])) == 3
     assert lib.isa_coarse_residual_backward(*(args[:8] + [a + 2] + args[9:])) == 1
+
+
+def test_static_status_query_rejected_on_host(isa):
+    """isa_forward_static_status refuses a NULL destination and a device on
+    which isa_forward_static has not run, before any CUDA call."""
+    lib = isa.load_library()
+    assert lib.isa_forward_static_status(0, None, None) == isa.ISA_ERR_INVALID_ARG
+    assert b"dst is NULL" in lib.isa_last_error()
+    word = ctypes.c_int32(-1)
+    assert lib.isa_forward_static_status(63, ctypes.addressof(word), None) == isa.ISA_ERR_INVALID_ARG
+    assert b"has not run" in lib.isa_last_error()
+    assert lib.isa_forward_static_status(-1, ctypes.addressof(word), None) == isa.ISA_ERR_INVALID_ARG
+    assert word.value == -1

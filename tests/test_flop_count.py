@@ -1,4 +1,4 @@
-"""The executed-work count behind the bench's TFLOP/s (`executed_flops`).
+"""The executed-work count behind the bench's TFLOP/s (`bench.executed_flops`).
 
 Convention (the ISA forward metric): 4*D FLOPs per (valid query token, key
 column) pair, where an exactly attended key token is one column and a pooled
@@ -10,6 +10,7 @@ import numpy as np
 import torch
 
 import block_sparse_attention_coarse_b200 as isa
+from bench import executed_flops
 import oracle as O
 from parity import oracle_params
 from workloads import Workload, bf16_to_f64, generate_bits
@@ -48,7 +49,7 @@ def test_count_matches_a_block_loop_with_partial_blocks():
     plans = [O.plan_head(bf16_to_f64(qb[h]), bf16_to_f64(kb[h]), bf16_to_f64(vb[h]), op) for h in range(w.BH)]
     assert any(c != w.block for c in plans[0].counts)
     p = isa.make_params(w.B, w.H, w.D, w.L_src, w.L_ctx, w.block, w.alpha_s, w.alpha_f, w.alpha_ns)
-    got = isa.executed_flops(p, fake_view(plans, plans[0].exact.shape[1]))
+    got = executed_flops(p, fake_view(plans, plans[0].exact.shape[1]))
     assert got == float(block_loop_count(plans, w.D))
 
 
@@ -68,4 +69,4 @@ def test_count_at_the_bench_shape_is_the_closed_form():
                                 None, kept, None, sharp, flat, exact))
     p = isa.make_params(2, 40, 128, 16384, 16384)
     per_head = (256 * 64 * 288 * 64 + 256 * 64 * (18 * 64 + 270)) * 4 * 128 + 2 * 512 * 512 * 128
-    assert isa.executed_flops(p, fake_view(plans, 18)) == float(80 * per_head) == 13.32916256768e12
+    assert executed_flops(p, fake_view(plans, 18)) == float(80 * per_head) == 13.32916256768e12

@@ -14,15 +14,16 @@ is then within a few u of the sum of the magnitudes of its terms, and since
 the logit gradients of a row add up to zero (cancellation) that sum is
 bounded by the tensor's scale rather than by the element.  Per head and
 gradient:  max |gpu - ref| <= 16u max|ref|  and  mean |gpu - ref| <= 4u rms(ref).
-Heads whose GPU plan differs from the oracle's (allowed within the planning
-margins) are excluded and counted; at most 10 % of the compared heads may be.
+Where the GPU plan differs from the oracle's inside the planning margins
+(both are then valid plans), the oracle's backward runs on the GPU's
+validated index sets, so every head is compared.
 """
 import numpy as np
 import pytest
 import torch
 
 import oracle as O
-from parity import check_head_plan, oracle_params, plan_view_host, to_torch_bf16
+from parity import check_head_plan, oracle_params, plan_from_gpu, plan_view_host, to_torch_bf16
 from workloads import Workload, bf16_to_f64, dout_head_bits, generate_bits, generate_dout_bits, head_bits, \
     named_workloads
 
@@ -56,10 +57,13 @@ def run_gpu(isa, w: Workload, qb, kb, vb, db):
     return grads, view
 
 
-def plan_identical(pl, view, h) -> bool:
+def gpu_plan(pl, view, h):
+    """The oracle plan with the GPU's index sets, once they pass the margin
+    rules (where the two plans differ only between near-equal scores, both
+    are valid and the gradients are compared for the GPU's choice)."""
     r = check_head_plan(pl, view, h)
     assert not r.errors, (h, r.errors[:5])
-    return r.ctx_equal and not r.split_moved and not r.exact_moved
+    return plan_from_gpu(pl, view, h)
 
 
 def assert_grads_close(got, ref, what):
@@ -95,14 +99,9 @@ def test_backward_matches_oracle(isa, name, B, H, D, Ls, Lc, b, a_s, a_f, a_ns):
     db = generate_dout_bits(w)
     (gq, gk, gv), view = run_gpu(isa, w, qb, kb, vb, db)
     op = oracle_params(w)
-    compared = excluded = 0
     for h in range(w.BH):
         qh, kh, vh, dh = (bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb, db))
-        pl = O.plan_head(qh, kh, vh, op)
-        if not plan_identical(pl, view, h):
-            excluded += 1
-            continue
-        compared += 1
+        pl = gpu_plan(O.plan_head(qh, kh, vh, op), view, h)
         ref = O.backward_head(qh, kh, vh, pl, op, dh)
         assert_grads_close((gq[h], gk[h], gv[h]), ref, (name, h))
         # context blocks the pre-selection dropped get exactly zero
@@ -110,7 +109,6 @@ def test_backward_matches_oracle(isa, name, B, H, D, Ls, Lc, b, a_s, a_f, a_ns):
         for c in dropped:
             rows = slice(Ls + c * b, min(Ls + (c + 1) * b, w.L))
             assert not gk[h][rows].any() and not gv[h][rows].any()
-    assert excluded <= 0.1 * (compared + excluded), (compared, excluded)
 
 
 def test_autograd_function_gradients(isa):
@@ -153,8 +151,7 @@ def test_backward_full_size(isa):
     op = oracle_params(w)
     q, k, v = (bf16_to_f64(x) for x in head_bits(w, h))
     dh = bf16_to_f64(dout_head_bits(w, h))
-    pl = O.plan_head(q, k, v, op)
-    assert plan_identical(pl, view, h)
+    pl = gpu_plan(O.plan_head(q, k, v, op), view, h)
     ref = O.backward_head(q, k, v, pl, op, dh)
     assert_grads_close((gq[h], gk[h], gv[h]), ref, ("dit14b", h))
 
@@ -199,9 +196,8 @@ def test_backward_timeout_path_reports_status_and_context_survives(isa):
     op = oracle_params(w)
     for h in range(w.BH):
         qh, kh, vh, dh = (bf16_to_f64(x.reshape(w.BH, w.L, w.D)[h]) for x in (qb, kb, vb, db))
-        pl = O.plan_head(qh, kh, vh, op)
-        if plan_identical(pl, view, h):
-            assert_grads_close((gq[h], gk[h], gv[h]), O.backward_head(qh, kh, vh, pl, op, dh), ("bto", h))
+        pl = gpu_plan(O.plan_head(qh, kh, vh, op), view, h)
+        assert_grads_close((gq[h], gk[h], gv[h]), O.backward_head(qh, kh, vh, pl, op, dh), ("bto", h))
 
 
 @pytest.mark.parametrize("name", ["long65k_b32", "sweep_L131072_D64"])
@@ -224,18 +220,13 @@ def test_backward_long_sequences(isa, name):
         assert np.all(np.abs(sv - dsum[h]) <= 4 * U * np.abs(gv[h]).astype(np.float64).sum(axis=0) + 1e-3), h
         assert np.all(np.abs(sk) <= 4 * U * np.abs(gk[h]).astype(np.float64).sum(axis=0) + 1e-3), h
     op = oracle_params(w)
-    checked = 0
     for h in (0, 23, 37):
         q, k, v = (bf16_to_f64(x) for x in head_bits(w, h))
         dh = bf16_to_f64(dout_head_bits(w, h))
-        pl = O.plan_head(q, k, v, op)
-        if not plan_identical(pl, view, h):
-            continue
-        checked += 1
+        pl = gpu_plan(O.plan_head(q, k, v, op), view, h)
         blocks = [int(pl.sharp[0]), int(pl.sharp[-1]), int(pl.flat[0]), int(pl.flat[len(pl.flat) // 2])]
         ref_dq, _, _ = O.backward_head(q, k, v, pl, op, dh, blocks=blocks)
         rows = np.concatenate([np.arange(pl.starts[i], pl.starts[i] + pl.counts[i]) for i in blocks])
         e = np.abs(gq[h][rows] - ref_dq[rows])
         r = ref_dq[rows]
         assert e.max() <= MAX_REL * np.abs(r).max() and e.mean() <= MEAN_REL * np.sqrt((r ** 2).mean()), (name, h)
-    assert checked >= 2, checked

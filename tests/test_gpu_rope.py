@@ -9,9 +9,9 @@
     rope (rounded once to bf16, the precision the GPU hands on) -> plan ->
     forward.  The two sides plan from rotations rounded independently (a few
     elements one bf16 ulp apart), so value checks allow one rounding of the
-    inputs, blocks whose plan decisions differ are excluded from the output
-    comparison and counted (at most 5 %), and outputs meet the tolerances of
-    the other parity tests.
+    inputs and index sets that differ beyond the margins are counted (at most
+    5 %); every block's output is compared with the oracle run on the GPU's
+    plan, within the tolerances of the other parity tests.
 """
 import numpy as np
 import pytest
@@ -19,7 +19,7 @@ import torch
 
 import oracle as O
 from parity import (OUT_MAX_ABS, OUT_MEAN_ABS, block_rows, check_head_plan, compare_outputs, oracle_params,
-                    plan_view_host, to_torch_bf16)
+                    plan_from_gpu, plan_view_host, to_torch_bf16)
 from workloads import Workload, bf16_to_f64, f32_to_bf16_bits, generate_bits, named_workloads
 
 pytestmark = pytest.mark.gpu
@@ -111,7 +111,7 @@ def test_isa_with_rope_end_to_end(isa, name, B, H, D, Ls, Lc, b):
     out = out.float().cpu().numpy().reshape(w.BH, w.L, D)
     lse = lse.cpu().numpy().reshape(w.BH, w.L)
     op = oracle_params(w)
-    n_rows = n_moved = 0
+    n_sets = n_outside = 0
     for h in range(w.BH):
         # oracle side: its own rotation of the bf16 inputs, rounded once to bf16
         qo = O.rope_decoupled(bf16_to_f64(qb.reshape(w.BH, w.L, D)[h]), Ls, Lc)
@@ -121,16 +121,14 @@ def test_isa_with_rope_end_to_end(isa, name, B, H, D, Ls, Lc, b):
         pl = O.plan_head(qo, ko, vo, op)
         r = check_head_plan(pl, view, h, inputs_equal=False)
         assert not r.errors, (h, r.errors[:5])
-        if not r.ctx_equal:
-            n_moved += pl.T
-            continue
-        moved = set(r.split_moved) | set(r.exact_moved)
-        use = [i for i in range(pl.T) if i not in moved]
-        n_moved += pl.T - len(use)
-        n_rows += pl.T
-        ref, ref_lse = O.forward_head(qo, ko, vo, pl, op, blocks=use)
-        rows = block_rows(pl, use)
+        # the plans came from inputs one bf16 rounding apart, so an index set
+        # may differ beyond the margin where scores are that close: count such
+        # sets, then compare every block with the oracle run on the GPU's plan
+        n_outside += len(r.outside_margin)
+        n_sets += 1 + (pl.T > len(pl.sharp)) + len(pl.flat)
+        ref, ref_lse = O.forward_head(qo, ko, vo, plan_from_gpu(pl, view, h), op)
+        rows = block_rows(pl, range(pl.T))
         mx, mean = compare_outputs(out[h], ref, rows)
         assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (h, mx, mean)
         assert np.abs(lse[h][rows] - ref_lse[rows]).max() <= 2e-2
-    assert n_moved <= 0.05 * max(n_rows, 1), (n_moved, n_rows)
+    assert n_outside <= 0.05 * max(n_sets, 1), (n_outside, n_sets)

@@ -78,8 +78,8 @@ def named_workloads() -> Dict[str, Workload]:
     long65k  : clustered, B=1 H=40 D=128, 32768 + 32768 tokens, b=64 (the
                b=32 and alpha_f variants are built with ``replace``).
     sweep*   : clustered, B=1 H=40, total length 4096..131072 split evenly;
-               at 131072 tokens, D=128 also alpha_s 0.0625 / 0.25 and
-               alpha_ns 0.03125 / 0.125 (the ratio grid).
+               at 131072 tokens, D=128 also the ratio grid alpha_s in
+               {0.0625, 0.125, 0.25} x alpha_ns in {0.03125, 0.0625, 0.125}.
     """
     w = {
         "tiny": Workload("tiny", 1, 2, 64, 1024, 1024, kind="iid", seed=0),
@@ -96,9 +96,16 @@ def named_workloads() -> Dict[str, Workload]:
             name = f"sweep_L{total}_D{D}"
             w[name] = Workload(name, 1, 40, D, total // 2, total // 2, seed=4000 + point)
             point += 1
-    # the ratio grid at 131072 tokens, D=128 (alpha_s and alpha_ns moved one at a time)
+    # the ratio grid at 131072 tokens, D=128: alpha_s in {0.0625, 0.125, 0.25}
+    # x alpha_ns in {0.03125, 0.0625, 0.125} (the centre point is
+    # sweep_L131072_D128); the points on the centre's row and column first,
+    # then the four corners
     for tag, kw in (("as0625", dict(alpha_s=0.0625)), ("as25", dict(alpha_s=0.25)),
-                    ("ans03125", dict(alpha_ns=0.03125)), ("ans125", dict(alpha_ns=0.125))):
+                    ("ans03125", dict(alpha_ns=0.03125)), ("ans125", dict(alpha_ns=0.125)),
+                    ("as0625_ans03125", dict(alpha_s=0.0625, alpha_ns=0.03125)),
+                    ("as0625_ans125", dict(alpha_s=0.0625, alpha_ns=0.125)),
+                    ("as25_ans03125", dict(alpha_s=0.25, alpha_ns=0.03125)),
+                    ("as25_ans125", dict(alpha_s=0.25, alpha_ns=0.125))):
         name = f"sweep_L131072_D128_{tag}"
         w[name] = Workload(name, 1, 40, 128, 65536, 65536, seed=4000 + point, **kw)
         point += 1
