@@ -409,6 +409,43 @@ def run_gpu(args, w: Workload):
         torch.cuda.synchronize(dev)
         dense_ms = e0.elapsed_time(e1) / nd
 
+    # decoupled RoPE ahead of the plan: the standalone rotation pass then
+    # isa_plan, against the rotation folded into the pooling pass
+    # (isa_plan_rope), on the same inputs.  Algorithmic HBM bytes, N = the
+    # elements of one of Q, K, V: separate = rope (read Q, K + write Q, K) +
+    # pooling (read Q, K, V) = 14 N; fused = read Q, K, V + write Q, K = 10 N.
+    rope_leg = None
+    if not args.skip_rope:
+        qr, kr = torch.empty_like(q), torch.empty_like(k)
+        rws = torch.empty(isa.rope_workspace_size(p), dtype=torch.uint8, device=dev)
+        ws2 = isa.alloc_workspace(p, dev)
+
+        def separate():
+            isa.rope(q, k, p, ws=rws, q_out=qr, k_out=kr)
+            isa.plan(qr, kr, v, p, ws2)
+
+        def fused():
+            isa.plan_rope(q, k, v, p, ws=ws2, rope_ws=rws, q_rot=qr, k_rot=kr)
+
+        nr = max(3, min(args.steps, 10))
+        times = {}
+        for name, fn in (("separate", separate), ("fused", fused)):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(nr):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times[name] = e0.elapsed_time(e1) / nr
+        n_el = q.numel()
+        rope_leg = {"separate_ms": times["separate"], "fused_ms": times["fused"],
+                    "what": "isa_rope + isa_plan vs isa_plan_rope (RoPE folded into the pooling pass), base 10000",
+                    "hbm_bytes_separate": 14 * n_el, "hbm_bytes_fused": 10 * n_el,
+                    "hbm_bytes_saved": 4 * n_el}
+        del qr, kr, rws, ws2
+
     # the backward (isa_backward) on the same plan: dq, dk, dv of sum(dout * out)
     bwd = None
     if not args.skip_backward:
@@ -531,6 +568,8 @@ def run_gpu(args, w: Workload):
         line["e2e"] = e2e
     if bwd:
         line["backward"] = bwd
+    if rope_leg:
+        line["rope"] = rope_leg
     if long_ctx:
         line["long_context"] = long_ctx
     if world == 1 and not args.skip_cpu:
@@ -553,6 +592,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-coarse", action="store_true")
+    ap.add_argument("--skip-rope", action="store_true", help="skip the decoupled-RoPE leg")
     ap.add_argument("--skip-long", action="store_true", help="skip the 131072-token forward leg")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N>1: replicas = every rank runs the whole workload (weak scaling); "

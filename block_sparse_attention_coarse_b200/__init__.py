@@ -37,7 +37,7 @@ ISA_ERR_DEVICE_TIMEOUT = 5
 
 # every entry point declared in include/isa.h
 EXPORTS = (
-    "isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
+    "isa_plan_workspace_size", "isa_plan", "isa_plan_rope", "isa_plan_view_get", "isa_forward", "isa_dense",
     "isa_last_error", "isa_version", "isa_set_wait_timeout_ns", "isa_set_fault_injection",
     "isa_forward_static", "isa_forward_static_status", "isa_rope_workspace_size", "isa_rope", "isa_backward_workspace_size", "isa_backward",
     "isa_coarse_residual", "isa_coarse_residual_backward_workspace_size", "isa_coarse_residual_backward",
@@ -86,6 +86,7 @@ def load_library() -> ctypes.CDLL:
     vp, sz = ctypes.c_void_p, ctypes.c_size_t
     lib.isa_plan_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.isa_plan.argtypes = [P, vp, vp, vp, vp, sz, vp]
+    lib.isa_plan_rope.argtypes = [P, ctypes.c_float, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]
     lib.isa_plan_view_get.argtypes = [P, vp, sz, ctypes.POINTER(_PlanView)]
     lib.isa_forward.argtypes = [P, vp, vp, vp, vp, sz, vp, vp, vp]
     lib.isa_dense.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
@@ -104,7 +105,8 @@ def load_library() -> ctypes.CDLL:
     lib.isa_coarse_residual.argtypes = [P, ctypes.c_float, vp, sz, vp, vp]
     lib.isa_coarse_residual_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     lib.isa_coarse_residual_backward.argtypes = [P, ctypes.c_float, vp, sz, vp, vp, vp, vp, vp, vp, sz, vp]
-    for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_view_get", "isa_forward", "isa_dense",
+    for name in ("isa_plan_workspace_size", "isa_plan", "isa_plan_rope", "isa_plan_view_get", "isa_forward",
+                 "isa_dense",
                  "isa_set_wait_timeout_ns", "isa_set_fault_injection", "isa_rope_workspace_size", "isa_rope",
                  "isa_backward_workspace_size", "isa_backward", "isa_coarse_residual",
                  "isa_coarse_residual_backward_workspace_size", "isa_coarse_residual_backward"):
@@ -162,6 +164,30 @@ def plan(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optio
     _check(load_library().isa_plan(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), ws.data_ptr(),
                                    ws.numel(), _stream(stream)))
     return ws
+
+
+def plan_rope(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, base: float = 10000.0,
+              ws: Optional[torch.Tensor] = None, inplace: bool = False, rope_ws: Optional[torch.Tensor] = None,
+              stream=None, q_rot: Optional[torch.Tensor] = None, k_rot: Optional[torch.Tensor] = None):
+    """Decoupled RoPE of q and k folded into the planning pass (isa_plan_rope);
+    returns (ws, q_rot, k_rot): the plan and the rotated q and k that
+    `forward` takes with v.  q_rot, k_rot are the given tensors, q / k when
+    `inplace`, else new tensors."""
+    _check_qkv(q, k, v, p)
+    if ws is None:
+        ws = alloc_workspace(p, q.device)
+    if inplace:
+        qo, ko = q, k
+    else:
+        qo = torch.empty_like(q) if q_rot is None else q_rot
+        ko = torch.empty_like(k) if k_rot is None else k_rot
+        _check_qkv(qo, ko, ko, p)
+    if rope_ws is None:
+        rope_ws = torch.empty(rope_workspace_size(p), dtype=torch.uint8, device=q.device)
+    _check(load_library().isa_plan_rope(ctypes.byref(p), float(base), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        qo.data_ptr(), ko.data_ptr(), ws.data_ptr(), ws.numel(), rope_ws.data_ptr(),
+                                        rope_ws.numel(), _stream(stream)))
+    return ws, qo, ko
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ws: torch.Tensor, p: Params,
@@ -229,12 +255,18 @@ def rope_workspace_size(p: Params) -> int:
 
 
 def rope(q: torch.Tensor, k: torch.Tensor, p: Params, base: float = 10000.0, inplace: bool = False,
-         ws: Optional[torch.Tensor] = None, stream=None):
+         ws: Optional[torch.Tensor] = None, stream=None, q_out: Optional[torch.Tensor] = None,
+         k_out: Optional[torch.Tensor] = None):
     """Decoupled rotary position embedding of q and k (positions restart at 0
-    in the context segment); returns the rotated (q, k), new tensors unless
-    `inplace`."""
+    in the context segment); returns the rotated (q, k): q_out / k_out when
+    given, q / k when `inplace`, else new tensors."""
     _check_qkv(q, k, k, p)
-    qo, ko = (q, k) if inplace else (torch.empty_like(q), torch.empty_like(k))
+    if inplace:
+        qo, ko = q, k
+    else:
+        qo = torch.empty_like(q) if q_out is None else q_out
+        ko = torch.empty_like(k) if k_out is None else k_out
+        _check_qkv(qo, ko, ko, p)
     if ws is None:
         ws = torch.empty(rope_workspace_size(p), dtype=torch.uint8, device=q.device)
     _check(load_library().isa_rope(ctypes.byref(p), float(base), q.data_ptr(), k.data_ptr(), qo.data_ptr(),
@@ -347,8 +379,8 @@ def _copy_streams(dev: torch.device):
 def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, ws: Optional[torch.Tensor] = None,
                   device=None, rope_base: Optional[float] = None, out: Optional[torch.Tensor] = None,
                   chunks: int = 8) -> torch.Tensor:
-    """The user-level call: plan + forward, after the decoupled RoPE of q and
-    k when `rope_base` is given.
+    """The user-level call: plan + forward, with the decoupled RoPE of q and
+    k folded into the planning pass when `rope_base` is given.
 
     CUDA inputs stay on the device (returns a new device tensor).  CPU
     inputs (pinned, [B, H, L, D] bf16) are processed in `chunks` contiguous
@@ -360,8 +392,9 @@ def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, 
     synchronising it makes `out` complete."""
     if q.is_cuda:
         if rope_base is not None:
-            q, k = rope(q, k, p, rope_base)
-        ws = plan(q, k, v, p, ws)
+            ws, q, k = plan_rope(q, k, v, p, rope_base, ws)
+        else:
+            ws = plan(q, k, v, p, ws)
         return forward(q, k, v, ws, p)
     dev = torch.device(device or "cuda")
     if dev.index is None:
@@ -398,8 +431,9 @@ def isa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Params, 
             t.record_stream(compute)
         with torch.cuda.stream(compute):
             if rope_base is not None:
-                qd, kd = rope(qd, kd, pc, rope_base, inplace=True)
-            plan(qd, kd, vd, pc, ws)
+                plan_rope(qd, kd, vd, pc, rope_base, ws, inplace=True)
+            else:
+                plan(qd, kd, vd, pc, ws)
             od = forward(qd, kd, vd, ws, pc)
             done = torch.cuda.Event()
             done.record(compute)

@@ -276,6 +276,33 @@ isa_status isa_plan(const isa_params* p, const void* q, const void* k, const voi
   return ISA_OK;
 }
 
+isa_status isa_plan_rope(const isa_params* p, float base, const void* q, const void* k, const void* v, void* q_rot,
+                         void* k_rot, void* ws, size_t ws_bytes, void* rope_ws, size_t rope_ws_bytes, void* stream) {
+  Dims d;
+  isa_status s = make_dims(p, &d);
+  if (s != ISA_OK) return s;
+  if (!(base > 1.f) || !std::isfinite(base)) return fail(ISA_ERR_INVALID_ARG, "base must be finite and > 1");
+  if ((s = check_ptr(q, "q", 16)) != ISA_OK || (s = check_ptr(k, "k", 16)) != ISA_OK ||
+      (s = check_ptr(v, "v", 16)) != ISA_OK || (s = check_ptr(q_rot, "q_rot", 16)) != ISA_OK ||
+      (s = check_ptr(k_rot, "k_rot", 16)) != ISA_OK || (s = check_ptr(ws, "workspace", 256)) != ISA_OK ||
+      (s = check_ptr(rope_ws, "rope workspace", 16)) != ISA_OK)
+    return s;
+  const PlanLayout L = make_layout(d);
+  if (ws_bytes < L.total) return fail(ISA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  const size_t need = rope_table_bytes(d);
+  if (rope_ws_bytes < need) return fail(ISA_ERR_WORKSPACE, "rope workspace has %zu bytes, needs %zu", rope_ws_bytes, need);
+  if ((s = ensure_init()) != ISA_OK || (s = bind_device_of(q, "q")) != ISA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const PlanPtrs pp = make_ptrs(L, ws);
+  cudaError_t e = cudaMemsetAsync(pp.status, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  if ((e = launch_rope_table(d, (double)base, rope_ws, st)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+  const RopeArgs ra{static_cast<const float2*>(rope_ws), q_rot, k_rot};
+  e = launch_plan(d, q, k, v, pp, st, &ra);
+  if (e != cudaSuccess) return cuda_fail(e, "planning launch");
+  return ISA_OK;
+}
+
 // Sizes, plan pointers and work-list counts of the attention kernels (mode 0:
 // ISA items from the plan; mode 1: dense items).
 static AttnArgs attn_args(const Dims& d, int mode, const PlanPtrs* pp) {

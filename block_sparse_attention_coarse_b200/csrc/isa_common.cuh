@@ -74,9 +74,17 @@ struct BwdArgs {
   int kv_total;                // BH * kv_tiles
 };
 
+// Decoupled RoPE folded into the pooling pass (isa_plan_rope): the (cos, sin)
+// table and where the rotated Q and K rows go.
+struct RopeArgs {
+  const float2* tab;   // [max(L_src, L_ctx), D/2] (cos, sin) per segment position and pair
+  void* q_rot;         // bf16 [BH*L, D]; may be q (in place)
+  void* k_rot;         // bf16 [BH*L, D]; may be k (in place)
+};
+
 // launchers (host)
 cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
-                        cudaStream_t st);
+                        cudaStream_t st, const RopeArgs* rope = nullptr);
 cudaError_t launch_attention(int D, int R, const CUtensorMap* maps, const AttnArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_backward(const Dims& d, const CUtensorMap* maps, BwdArgs& b, int sm_count, cudaStream_t st);
 size_t coarse_backward_bytes(const Dims& d);
@@ -85,6 +93,7 @@ cudaError_t launch_coarse(const Dims& d, const PlanPtrs& pp, float gamma, void* 
 size_t rope_table_bytes(const Dims& d);
 cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
                         int sm_count, cudaStream_t st);
+cudaError_t launch_rope_table(const Dims& d, double base, void* tab, cudaStream_t st);
 void set_last_error(const char* msg);
 isa_status bind_device_of(const void* ptr, const char* name);
 
@@ -477,6 +486,19 @@ __device__ inline void warp_topk(const float* key, int n, int k, int* out, uint3
     base += __popc(selm);
     eq_seen += __popc(eqm);
   }
+}
+
+// One RoPE pair (2i, 2i+1) of bf16 values rotated by the angle whose
+// (cos, sin) is cs, in fp32, rounded once to bf16 (nearest even).  The
+// standalone rotation and the pooling pass share it, so both give the same
+// bits.
+__device__ __forceinline__ uint32_t rot_pair(uint32_t xv, float2 cs) {
+  const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&xv);
+  const float x0 = __low2float(x), x1 = __high2float(x);
+  const float y0 = fmaf(x0, cs.x, -x1 * cs.y);
+  const float y1 = fmaf(x0, cs.y, x1 * cs.x);
+  const __nv_bfloat162 y = __floats2bfloat162_rn(y0, y1);
+  return *reinterpret_cast<const uint32_t*>(&y);
 }
 
 // Token span of block `id` (source blocks first, each segment blocked on its own).

@@ -175,6 +175,17 @@ __device__ __forceinline__ void tmem_ld16x2_sync1(uint32_t t0, uint32_t (&r0)[32
       : "r"(t0), "n"(SPLIT)
       : "memory");
 }
+// One 16-column group (thread t < 16: columns [c, c+16), t >= 16:
+// [c+SPLIT, c+SPLIT+16)) and the wait:
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld16x2_sync1_16(uint32_t t0, uint32_t (&r0)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ISA_R16(r0)
+      : "r"(t0), "n"(SPLIT)
+      : "memory");
+}
 // Two groups and the wait:
 template <int SPLIT>
 __device__ __forceinline__ void tmem_ld16x2_sync2(uint32_t t0, uint32_t (&r0)[32], uint32_t t1, uint32_t (&r1)[32]) {
@@ -206,6 +217,21 @@ __device__ __forceinline__ void tmem_ld16x2_sync4(uint32_t t0, uint32_t (&r0)[32
       : ISA_R32(r0), ISA_R32(r1), ISA_R32(r2), ISA_R32(r3)
       : "r"(t0), "r"(t1), "r"(t2), "r"(t3), "n"(SPLIT)
       : "memory");
+}
+// Stores of 16 and 8 columns in the same split layout.
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};" ::
+          "r"(taddr),
+      "n"(SPLIT), ISA_W16(r)
+      : "memory");
+}
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st16x2_8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9};" ::"r"(taddr), "n"(SPLIT),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 template <int SPLIT>
 __device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const uint32_t (&r)[32]) {

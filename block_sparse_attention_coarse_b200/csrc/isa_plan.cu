@@ -4,6 +4,7 @@
 // In-Context Sparse Attention".
 //
 //   pool_kernel        step (1): per-segment blocks, fp32 means of Q, K, V
+//                      (optionally after the decoupled RoPE of Q and K)
 //   ctx_select_kernel  step (2): context importance (source query rows summed
 //                      over the source x context region of S), TopK, kept
 //                      list, bf16 pooled K/V of the kept blocks
@@ -21,12 +22,16 @@ namespace isa {
 // K1: pooling.  grid (T, BH, 3), 256 threads.  Each thread reads 16-byte
 // vectors (8 bf16) of D/8-wide row chunks; rows of the block are split over
 // 256/(D/8) row groups, reduced through shared memory.  HBM bound.
+// ROPE: the Q and K rows are first rotated (decoupled RoPE, rot_pair with the
+// (cos, sin) of the token's segment position), written once to q_rot/k_rot
+// for the attention, and pooled from those rounded values, so Q and K are
+// read once for both steps.  Each vector is read and written by one thread,
+// so q_rot/k_rot may be q/k; plain loads then (not the read-only path).
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                   const __nv_bfloat16* __restrict__ k,
-                                                   const __nv_bfloat16* __restrict__ v, Dims dm, float* Qc,
-                                                   float* Kc, float* Vc) {
+template <int D, bool ROPE>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                                   const __nv_bfloat16* v, Dims dm, float* Qc, float* Kc,
+                                                   float* Vc, RopeArgs rope) {
   constexpr int CH = D / 8;          // 16-byte chunks per row
   constexpr int RG = 256 / CH;       // row groups
   __shared__ float part[RG][D];
@@ -35,16 +40,40 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   float* out = which == 0 ? Qc : (which == 1 ? Kc : Vc);
   const int2 sp = block_span(blk, dm.L_src, dm.L_ctx, dm.b, dm.T_src);
   const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
-  const uint4* base = reinterpret_cast<const uint4*>(X + ((size_t)bh * dm.L + sp.x) * D) + ch;
+  const size_t first = ((size_t)bh * dm.L + sp.x) * CH + ch;   // this thread's vector of the block's row 0
+  const uint4* base = reinterpret_cast<const uint4*>(X) + first;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   constexpr int MAXR = 64 / RG > 0 ? 64 / RG : 1;   // rows per thread for b <= 64
   uint4 buf[MAXR];
+  const bool rot = ROPE && which < 2;
 #pragma unroll
   for (int i = 0; i < MAXR; ++i) {
     const int r = rg + i * RG;
-    buf[i] = r < sp.y ? __ldg(base + (size_t)r * CH) : make_uint4(0, 0, 0, 0);
+    if constexpr (ROPE) {
+      buf[i] = r < sp.y ? base[(size_t)r * CH] : make_uint4(0, 0, 0, 0);
+    } else {
+      buf[i] = r < sp.y ? __ldg(base + (size_t)r * CH) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (rot) {
+    // segment position of the block's first token (blocks never straddle segments)
+    const int pos0 = blk < dm.T_src ? sp.x : sp.x - dm.L_src;
+    uint4* dst = reinterpret_cast<uint4*>(which == 0 ? rope.q_rot : rope.k_rot) + first;
+#pragma unroll
+    for (int i = 0; i < MAXR; ++i) {
+      const int r = rg + i * RG;
+      if (r < sp.y) {
+        const float4* tp = reinterpret_cast<const float4*>(rope.tab + (size_t)(pos0 + r) * (D / 2) + 4 * ch);
+        const float4 t01 = __ldg(tp), t23 = __ldg(tp + 1);
+        buf[i] = make_uint4(rot_pair(buf[i].x, make_float2(t01.x, t01.y)),
+                            rot_pair(buf[i].y, make_float2(t01.z, t01.w)),
+                            rot_pair(buf[i].z, make_float2(t23.x, t23.y)),
+                            rot_pair(buf[i].w, make_float2(t23.z, t23.w)));
+        dst[(size_t)r * CH] = buf[i];
+      }
+    }
   }
 #pragma unroll
   for (int i = 0; i < MAXR; ++i) {
@@ -386,11 +415,15 @@ static size_t exact_kernel_smem(const Dims& dm) {
 
 template <int D>
 static cudaError_t launch_plan_d(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
-                                 cudaStream_t st) {
-  pool_kernel<D><<<dim3(dm.T, dm.BH, 3), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
-                                                       reinterpret_cast<const __nv_bfloat16*>(k),
-                                                       reinterpret_cast<const __nv_bfloat16*>(v), dm, pp.Qc, pp.Kc,
-                                                       pp.Vc);
+                                 cudaStream_t st, const RopeArgs* rope) {
+  const dim3 pgrid(dm.T, dm.BH, 3);
+  const auto* qb = reinterpret_cast<const __nv_bfloat16*>(q);
+  const auto* kb = reinterpret_cast<const __nv_bfloat16*>(k);
+  const auto* vb = reinterpret_cast<const __nv_bfloat16*>(v);
+  if (rope)
+    pool_kernel<D, true><<<pgrid, 256, 0, st>>>(qb, kb, vb, dm, pp.Qc, pp.Kc, pp.Vc, *rope);
+  else
+    pool_kernel<D, false><<<pgrid, 256, 0, st>>>(qb, kb, vb, dm, pp.Qc, pp.Kc, pp.Vc, RopeArgs{});
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t sm_ctx = sizeof(float) * (D + dm.T_ctx) + sizeof(int) * dm.K_sel;
@@ -431,11 +464,11 @@ static cudaError_t prepare_plan_kernels() {
 }
 
 cudaError_t launch_plan(const Dims& dm, const void* q, const void* k, const void* v, const PlanPtrs& pp,
-                        cudaStream_t st) {
+                        cudaStream_t st, const RopeArgs* rope) {
   static std::atomic<unsigned long long> attr_done{0};
   const cudaError_t e = once_per_device(attr_done, prepare_plan_kernels);
   if (e != cudaSuccess) return e;
-  return dm.D == 64 ? launch_plan_d<64>(dm, q, k, v, pp, st) : launch_plan_d<128>(dm, q, k, v, pp, st);
+  return dm.D == 64 ? launch_plan_d<64>(dm, q, k, v, pp, st, rope) : launch_plan_d<128>(dm, q, k, v, pp, st, rope);
 }
 
 }  // namespace isa

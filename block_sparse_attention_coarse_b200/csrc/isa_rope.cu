@@ -11,7 +11,9 @@
 // Two launches: a table of (cos, sin) per (segment position, pair) computed
 // in double precision (max(L_src, L_ctx) * D/2 entries, a few MB, read back
 // from L2), then one streaming pass over Q and K (HBM-bound: every element
-// read once and written once).
+// read once and written once).  isa_plan_rope uses the same table and the
+// same rotation (rot_pair) inside the pooling pass instead of the second
+// launch, so Q and K are read once for both.
 #include <algorithm>
 
 #include "isa_common.cuh"
@@ -28,15 +30,6 @@ __global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ ta
   double s, c;
   sincos((double)pos * theta, &s, &c);
   tab[e] = make_float2((float)c, (float)s);
-}
-
-__device__ __forceinline__ uint32_t rot_pair(uint32_t xv, float2 cs) {
-  const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&xv);
-  const float x0 = __low2float(x), x1 = __high2float(x);
-  const float y0 = fmaf(x0, cs.x, -x1 * cs.y);
-  const float y1 = fmaf(x0, cs.y, x1 * cs.x);
-  const __nv_bfloat162 y = __floats2bfloat162_rn(y0, y1);
-  return *reinterpret_cast<const uint32_t*>(&y);
 }
 
 // One thread per 8 consecutive components (4 pairs) of one token row, for
@@ -63,12 +56,16 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const uint4* q, const u
 
 size_t rope_table_bytes(const Dims& d) { return (size_t)std::max(d.L_src, d.L_ctx) * (d.D / 2) * sizeof(float2); }
 
-cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
-                        int sm_count, cudaStream_t st) {
+cudaError_t launch_rope_table(const Dims& d, double base, void* tab, cudaStream_t st) {
   const int n_pos = std::max(d.L_src, d.L_ctx);
   const int n_tab = n_pos * (d.D / 2);
   rope_table_kernel<<<(n_tab + 255) / 256, 256, 0, st>>>(static_cast<float2*>(tab), n_pos, d.D, base);
-  cudaError_t e = cudaGetLastError();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope(const Dims& d, double base, const void* q, const void* k, void* qo, void* ko, void* tab,
+                        int sm_count, cudaStream_t st) {
+  cudaError_t e = launch_rope_table(d, base, tab, st);
   if (e != cudaSuccess) return e;
   const size_t n_vec = (size_t)d.BH * d.L * (d.D / 8);
   const size_t want = (n_vec + 255) / 256;

@@ -115,6 +115,25 @@ isa_status isa_plan_workspace_size(const isa_params* p, size_t* bytes);
 isa_status isa_plan(const isa_params* p, const void* q, const void* k, const void* v,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* isa_rope followed by isa_plan in one pass over Q and K: the decoupled
+ * RoPE of the techwalker.com article ("Decoupled RoPE": the reference
+ * video's positions restart at 0) and the summary card (innovation (d)),
+ * with the rotation, positions and rounding of isa_rope below, folded into
+ * the pooling of step (1).  The pooling kernel rotates each Q and K row as
+ * it reads it, writes the rotated bf16 row to q_rot / k_rot, and pools from
+ * those values; the results (q_rot, k_rot and the plan in ws) are bit for bit
+ * those of isa_rope then isa_plan, with Q and K read once instead of twice.
+ *   q, k, v      : device bf16 [B,H,L,D] (before the rotation)
+ *   q_rot, k_rot : device bf16 [B,H,L,D], every element written; may equal
+ *                  q, k (in place).  Give them, with v, to isa_forward.
+ *   base         : > 1 (10000 is the usual value)
+ *   ws           : the plan workspace, as for isa_plan
+ *   rope_ws      : device, >= isa_rope_workspace_size bytes, 16-byte aligned;
+ *                  caller-owned scratch for the (cos, sin) table
+ * Launches 7 kernels on `stream` (6 when no block is flat). */
+isa_status isa_plan_rope(const isa_params* p, float base, const void* q, const void* k, const void* v, void* q_rot,
+                         void* k_rot, void* ws, size_t ws_bytes, void* rope_ws, size_t rope_ws_bytes, void* stream);
+
 /* Fills `view` with the sizes of the plan for `p` and device pointers into
  * `ws` (no launch, no copy; contents valid once isa_plan has run). */
 isa_status isa_plan_view_get(const isa_params* p, const void* ws, size_t ws_bytes,

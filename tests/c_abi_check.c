@@ -24,7 +24,7 @@ typedef void (*any_fn)(void);
 
 int main(void) {
   const any_fn entry_points[] = {
-      (any_fn)isa_plan_workspace_size, (any_fn)isa_plan, (any_fn)isa_plan_view_get,
+      (any_fn)isa_plan_workspace_size, (any_fn)isa_plan, (any_fn)isa_plan_rope, (any_fn)isa_plan_view_get,
       (any_fn)isa_forward, (any_fn)isa_dense, (any_fn)isa_forward_static,
       (any_fn)isa_forward_static_status, (any_fn)isa_backward_workspace_size, (any_fn)isa_backward, (any_fn)isa_coarse_residual,
       (any_fn)isa_coarse_residual_backward_workspace_size, (any_fn)isa_coarse_residual_backward,

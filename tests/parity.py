@@ -171,7 +171,7 @@ def plan_from_gpu(pl: O.HeadPlan, gpu: dict, h: int) -> O.HeadPlan:
     coarse scores and token counts stay the oracle's fp64 values."""
     kept = gpu_kept(pl, gpu, h)
     flat = np.asarray(gpu["flat_ids"][h], np.int64)
-    exact = np.sort(np.asarray(gpu["exact"][h], np.int64).reshape(len(flat), -1), axis=1)
+    exact = np.sort(np.asarray(gpu["exact"][h], np.int64).reshape(len(flat), pl.exact.shape[1]), axis=1)
     return dataclasses.replace(pl, ctx_sel=np.sort(np.asarray(gpu["ctx_sel"][h], np.int64)), kept=kept,
                                sharp=np.asarray(gpu["sharp_ids"][h], np.int64), flat=flat, exact=exact)
 

@@ -5,7 +5,10 @@
     element must agree within two bf16 half-ulps of the oracle's value
     (|gpu - ref| <= 2^-8 |ref| + 1e-6).
   * In place and out of place give identical bits.
-  * End to end: rope -> isa_plan -> isa_forward on the GPU against the oracle's
+  * isa_plan_rope (the rotation inside the pooling pass) equals isa_rope then
+    isa_plan bit for bit: rotated q, k and every plan array.
+  * End to end: rope -> isa_plan -> isa_forward (and isa_plan_rope ->
+    isa_forward) on the GPU against the oracle's
     rope (rounded once to bf16, the precision the GPU hands on) -> plan ->
     forward.  The two sides plan from rotations rounded independently (a few
     elements one bf16 ulp apart), so value checks allow one rounding of the
@@ -94,16 +97,67 @@ def test_rope_full_size_sampled_heads(isa):
             assert_rotation_close(g[h], ref)
 
 
+def assert_plans_equal(isa, p, ws_a, ws_b):
+    va, vb = isa.plan_view(p, ws_a), isa.plan_view(p, ws_b)
+    for name, a in va.items():
+        if isinstance(a, torch.Tensor):
+            assert torch.equal(a, vb[name]), name
+
+
+@pytest.mark.parametrize("B,H,D,L_src,L_ctx,b,base", [(1, 2, 128, 520, 300, 64, 10000.0),
+                                                        (2, 2, 64, 333, 97, 32, 500.0),
+                                                        (1, 3, 128, 1000, 1, 64, 1e6)])
+def test_plan_rope_equals_rope_then_plan(isa, B, H, D, L_src, L_ctx, b, base):
+    """isa_plan_rope (the rotation folded into the pooling pass) gives bit
+    for bit the rotated q, k and the plan of isa_rope followed by isa_plan,
+    out of place and in place, and so the same forward output."""
+    w = Workload("plan_rope", B, H, D, L_src, L_ctx, block=b, alpha_s=0.25, alpha_f=0.5, alpha_ns=0.2, seed=64)
+    qb, kb, vb = generate_bits(w)
+    q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
+    p = params_of(isa, w)
+    qr, kr = isa.rope(q, k, p, base)
+    ws_sep = isa.plan(qr, kr, v, p)
+    ws_fused, qf, kf = isa.plan_rope(q, k, v, p, base)
+    q2, k2 = q.clone(), k.clone()
+    ws_ip, q2r, k2r = isa.plan_rope(q2, k2, v, p, base, inplace=True)
+    torch.cuda.synchronize()
+    assert torch.equal(qf, qr) and torch.equal(kf, kr)
+    assert q2r.data_ptr() == q2.data_ptr() and torch.equal(q2, qr) and torch.equal(k2, kr)
+    assert torch.equal(q, to_torch_bf16(qb)) and torch.equal(k, to_torch_bf16(kb))   # inputs untouched
+    assert_plans_equal(isa, p, ws_sep, ws_fused)
+    assert_plans_equal(isa, p, ws_sep, ws_ip)
+    assert int(isa.plan_view(p, ws_fused)["status"].item()) == 0
+    assert torch.equal(isa.forward(qr, kr, v, ws_sep, p), isa.forward(qf, kf, v, ws_fused, p))
+
+
+def test_plan_rope_equals_rope_then_plan_full_size(isa):
+    """The same bit-equality on every head of the bench shape (B=2, H=40,
+    16384 + 16384 tokens, D=128)."""
+    w = named_workloads()["dit14b"]
+    q, k, v = (to_torch_bf16(x) for x in generate_bits(w))
+    p = params_of(isa, w)
+    qr, kr = isa.rope(q, k, p)
+    ws_sep = isa.plan(qr, kr, v, p)
+    ws_fused, qf, kf = isa.plan_rope(q, k, v, p)
+    torch.cuda.synchronize()
+    assert torch.equal(qf, qr) and torch.equal(kf, kr)
+    assert_plans_equal(isa, p, ws_sep, ws_fused)
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["plan_rope", "rope_then_plan"])
 @pytest.mark.parametrize("name,B,H,D,Ls,Lc,b", [("rope_e2e", 1, 2, 128, 520, 300, 64),
                                                 ("rope_e2e_b32", 1, 2, 64, 333, 200, 32)])
-def test_isa_with_rope_end_to_end(isa, name, B, H, D, Ls, Lc, b):
+def test_isa_with_rope_end_to_end(isa, name, B, H, D, Ls, Lc, b, fused):
     w = Workload(name, B, H, D, Ls, Lc, block=b, alpha_s=0.25, alpha_f=0.5, alpha_ns=0.2, seed=63)
     qb, kb, vb = generate_bits(w)
     q, k, v = (to_torch_bf16(x) for x in (qb, kb, vb))
     p = params_of(isa, w)
     lse = torch.empty(B, H, w.L, dtype=torch.float32, device="cuda")
-    qr, kr = isa.rope(q, k, p)
-    ws = isa.plan(qr, kr, v, p)
+    if fused:
+        ws, qr, kr = isa.plan_rope(q, k, v, p)
+    else:
+        qr, kr = isa.rope(q, k, p)
+        ws = isa.plan(qr, kr, v, p)
     out = isa.forward(qr, kr, v, ws, p, lse=lse)
     torch.cuda.synchronize()
     view = plan_view_host(isa.plan_view(p, ws))

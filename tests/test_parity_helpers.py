@@ -8,7 +8,7 @@ import numpy as np
 
 import oracle as O
 from parity import (MARGIN_EXACT, block_rows, check_head_plan, compare_outputs, energy_from_oracle,
-                    oracle_params, topk_agrees)
+                    oracle_params, plan_from_gpu, topk_agrees)
 from workloads import Workload, bf16_to_f64, generate_bits
 
 
@@ -105,3 +105,72 @@ def test_compare_outputs_reads_only_the_listed_rows():
     mx, mean = compare_outputs(got, ref, rows)
     assert mx == 0.5 and abs(mean - 0.5 / (32 * 4)) < 1e-12
     assert compare_outputs(got, ref, np.zeros(0, np.int64)) == (0.0, 0.0)
+
+
+def view_of(pl):
+    """A one-head plan view (host arrays) holding an oracle plan's index sets."""
+    words = (len(pl.kept) + 31) // 32
+    bits = np.zeros((len(pl.flat), words), np.int64)
+    for r, row in enumerate(pl.exact):
+        for x in row:
+            bits[r, x // 32] |= 1 << (x % 32)
+    return {"Qc": pl.Qc[None].copy(), "Kc": pl.Kc[None].copy(), "Vc": pl.Vc[None].copy(), "imp": pl.imp[None].copy(),
+            "ctx_sel": pl.ctx_sel[None].copy(), "kept": pl.kept[None].copy(),
+            "energy": energy_from_oracle(pl)[None].copy(), "sharp_ids": pl.sharp[None].copy(),
+            "flat_ids": pl.flat[None].copy(), "exact": pl.exact[None].copy(), "exact_bits": bits[None]}
+
+
+def test_plan_from_gpu_round_trips_the_oracle_plan():
+    """Injecting a plan's own index sets gives back the same plan, and the
+    same output; also with no flat block (alpha_f = 0) and with no exact
+    block (alpha_ns = 0)."""
+    for a_f, a_ns in ((0.5, 0.25), (0.0, 0.25), (1.0, 0.0)):
+        w = Workload("inject", 1, 1, 64, 300, 200, block=32, alpha_s=0.5, alpha_f=a_f, alpha_ns=a_ns, seed=12)
+        qb, kb, vb = (bf16_to_f64(x.reshape(w.L, w.D)) for x in generate_bits(w))
+        op = oracle_params(w)
+        pl = O.plan_head(qb, kb, vb, op)
+        view = view_of(pl)
+        r = check_head_plan(pl, view, 0)
+        assert not r.errors and r.ctx_equal and not r.split_moved and not r.exact_moved
+        got = plan_from_gpu(pl, view, 0)
+        for name in ("ctx_sel", "kept", "sharp", "flat", "exact"):
+            assert np.array_equal(getattr(got, name), getattr(pl, name)), (a_f, a_ns, name)
+        o1, l1 = O.forward_head(qb, kb, vb, pl, op)
+        o2, l2 = O.forward_head(qb, kb, vb, got, op)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_plan_from_gpu_uses_the_gpu_choice():
+    """A within-margin exact-list swap in the CUDA plan: the check accepts it
+    and records the block as moved, and the injected plan carries the CUDA
+    choice, so the oracle's output for that block changes with it."""
+    w = Workload("inject2", 1, 1, 64, 300, 200, block=32, alpha_s=0.5, alpha_f=0.5, alpha_ns=0.25, seed=12)
+    qb, kb, vb = (bf16_to_f64(x.reshape(w.L, w.D)) for x in generate_bits(w))
+    op = oracle_params(w)
+    pl = O.plan_head(qb, kb, vb, op)
+    # move the first flat block's k-th exact block to the (k+1)-th, as a
+    # margin-sized fp32 disagreement would; widen the margin to accept it
+    b0 = int(pl.flat[0])
+    row = pl.S[b0, pl.kept]
+    order = np.lexsort((np.arange(len(row)), -row))
+    k = pl.exact.shape[1]
+    swapped = sorted((set(pl.exact[0].tolist()) - {int(order[k - 1])}) | {int(order[k])})
+    view = view_of(pl)
+    view["exact"][0][0] = swapped
+    view["exact_bits"][0][0] = 0
+    for x in swapped:
+        view["exact_bits"][0][0, x // 32] |= 1 << (x % 32)
+    import parity
+    old = parity.MARGIN_EXACT
+    parity.MARGIN_EXACT = float(row[order[k - 1]] - row[order[k]]) + 1e-9
+    try:
+        r = check_head_plan(pl, view, 0)
+    finally:
+        parity.MARGIN_EXACT = old
+    assert not r.errors and r.exact_moved == [b0]
+    got = plan_from_gpu(pl, view, 0)
+    assert got.exact[0].tolist() == swapped
+    o_ref, _ = O.forward_head(qb, kb, vb, pl, op, blocks=[b0])
+    o_got, _ = O.forward_head(qb, kb, vb, got, op, blocks=[b0])
+    rows = block_rows(pl, [b0])
+    assert not np.array_equal(o_ref[rows], o_got[rows])
