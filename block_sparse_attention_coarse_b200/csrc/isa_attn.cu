@@ -40,11 +40,6 @@ constexpr int kNSK = 3;             // K pipeline stages
 constexpr int kNSV = 2;             // V pipeline stages
 constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
 constexpr uint32_t kTmemO = 384;    // TMEM column of O (after three 128-column S buffers)
-// Exponentials of column pairs p with bit (p % 8) set go through the cubic on
-// the FMA pipe, the rest through MUFU.  All on MUFU measured fastest at both
-// D=128 and D=64 (the FMA and ALU pipes are the more contended ones here;
-// 1, 2, 3 and 4 pairs of 8 on the cubic were 1-6 % slower).
-constexpr uint32_t kPolyPairs = 0x00u;
 
 template <int D, int R>
 struct Cfg {
@@ -356,24 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
-          float2 pp;
-          if (kPolyPairs & (1u << ((c >> 1) & 7))) {
-            pp = ex2_poly2(x);             // FMA/ALU pipes
-          } else {
-            pp.x = ex2(x.x);               // MUFU
-            pp.y = ex2(x.y);
-          }
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));   // MUFU; 2^-inf = +0 for masked columns
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pp);
           pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
-        }
-        if (cur.masked) {
-          // the polynomial leaves masked columns at a denormal: clear them in P
-          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint32_t bits = ((e < 16 ? w0 : w1) >> ((2 * e) & 31)) & 3u;
-            pk[e] &= (bits & 1u ? 0x0000FFFFu : 0u) | (bits & 2u ? 0xFFFF0000u : 0u);
-          }
         }
         const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const float2 a03 = fadd2(a01, a23);

@@ -410,27 +410,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// 2^x for a pair of floats on the FMA/ALU pipes (no MUFU): x = n + f with
-// n = round(x), f in [-1/2, 1/2]; 2^f by a cubic with 7.5e-5 maximum relative
-// error (relative-minimax fit by Lawson's algorithm, see fit_exp2_poly.py);
-// 2^n by adding n to the exponent field.  x is clamped to [-126, 126]: very
-// negative inputs (and -inf) give a denormal below 1.2e-38 instead of 0, and
-// large ones saturate near 2^126 instead of wrapping the exponent field.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fminf(fmaxf(x.x, -126.f), 126.f);
-  x.y = fminf(fmaxf(x.y, -126.f), 126.f);
-  const float2 magic = make_float2(12582912.f, 12582912.f);   // 1.5 * 2^23
-  const float2 t = fadd2(x, magic);                              // n in the low mantissa bits
-  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(__uint_as_float(0x3D61FBAFu), __uint_as_float(0x3D61FBAFu)), f,
-                   make_float2(__uint_as_float(0x3E786F0Du), __uint_as_float(0x3E786F0Du)));
-  p = ffma2(p, f, make_float2(__uint_as_float(0x3F31798Du), __uint_as_float(0x3F31798Du)));
-  p = ffma2(p, f, make_float2(__uint_as_float(0x3F7FFB49u), __uint_as_float(0x3F7FFB49u)));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Order-preserving map of a float to an unsigned key.
 __device__ __forceinline__ uint32_t f2ord(float f) {
   uint32_t u = __float_as_uint(f);
