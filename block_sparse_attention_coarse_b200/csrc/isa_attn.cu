@@ -10,8 +10,10 @@
 //   sharp item : G sharp blocks of one head; KV tiles run over the kept
 //                blocks (source blocks, then the selected context blocks)
 //   flat item  : G flat blocks of one head; first n_exact tiles whose
-//                sub-block g is exact block j of query block g (block-diagonal
-//                mask), then the pooled tiles: 128 rows of the head's kept
+//                sub-block g is exact block j of query block g (block-diagonal:
+//                a softmax warp's rows, one query block, load and exponentiate
+//                only their own sub-block's columns and write zeros for the
+//                rest of P), then the pooled tiles: 128 rows of the head's kept
 //                pooled keys/values (Kp, Vp) with logit bias log2(n_j) and the
 //                row's own exact blocks masked out
 //   dense item : 128 consecutive query tokens against all L tokens
@@ -40,6 +42,11 @@ constexpr int kNSK = 3;             // K pipeline stages
 constexpr int kNSV = 2;             // V pipeline stages
 constexpr float kRescaleLog2 = 8.f; // lazy rescaling threshold (log2 units)
 constexpr uint32_t kTmemO = 384;    // TMEM column of O (after three 128-column S buffers)
+
+template <bool B>
+struct FlatTag {
+  static constexpr bool value = B;
+};
 
 template <int D, int R>
 struct Cfg {
@@ -293,98 +300,172 @@ __global__ void __launch_bounds__(kThreads, 1)
         jm1 = (a.L - 1) / 128;
       }
       int ekk = load_exact(a, I, 0, g_r);
-      for (int j = 0; j < I.ntiles; ++j, ++t) {
-        TileMeta cur;
-        if (I.kind == 2 || j == jm0 || j == jm1) {
-          cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
-          ekk = load_exact(a, I, j + 1, g_r);
-        } else {
-          cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
-          cur.pooled = 0;
-          cur.masked = 0;
-        }
-        const int buf = t % 3;
-        if (!s_ready && !__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t / 3) & 1, wc))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t sr[2][32];
-        // columns 64h + 0..31 and 64h + 32..63, waited for in the same statement
-        tmem_ld16x2_sync2<64>(trow + buf * 128, sr[0], trow + buf * 128 + 32, sr[1]);
-        float s[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-        if (cur.masked) {
-          const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = ((((c < 32) ? w0 : w1) >> (c & 31)) & 1u) ? s[c] : -INFINITY;
-          if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
-            const int kk0 = (j - a.n_exact) * 128 + 64 * h;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
+      // Two instances of the tile loop: flat items (with the block-diagonal
+      // exact tiles) and the rest, so the hot loop of sharp items carries no
+      // code of the other.
+      auto tile_loop = [&](auto flat_tag) {
+        constexpr bool FLAT = decltype(flat_tag)::value;
+        for (int j = 0; j < I.ntiles; ++j, ++t) {
+          // An exact tile of a flat item is block-diagonal: this warp's rows
+          // (one query block) take part only in the columns of their own
+          // sub-block, [g_r*R, g_r*R + dcnt).  Only those columns are loaded
+          // and exponentiated; P is zero elsewhere.
+          const bool diag = FLAT && j < a.n_exact;   // warp-uniform
+          int dcnt = R;
+          TileMeta cur;
+          if (diag) {
+            dcnt = kept_count(a, ic, ekk);
+            ekk = load_exact(a, I, j + 1, g_r);
+          } else if (FLAT || j == jm0 || j == jm1) {
+            cur = tile_meta<R, G>(a, I, ic, j, g_r, rbits, ekk);
+            ekk = load_exact(a, I, j + 1, g_r);
+          } else {
+            cur.mw[0] = cur.mw[1] = cur.mw[2] = cur.mw[3] = 0xFFFFFFFFu;
+            cur.pooled = 0;
+            cur.masked = 0;
           }
-        }
-        // half-row maximum: 8 independent chains of 3-input max
-        float mxa[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mxa[e] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
-        const float mh = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
-        const float bias = cur.pooled ? log2b : 0.f;
-        const float mx = fmaxf(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 16)) * sl2 + bias;   // whole row
-        const bool need = mx > m_run + kRescaleLog2;
-        const float m_new = need ? mx : m_run;
-        const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = need ? ex2(m_run - m_ref) : 1.f;
-        const float neg = bias - m_ref;
-        // Is S of the next tile (t+1, possibly the next item's first) there
-        // already?  The test's latency overlaps the exponentials below, and a
-        // set phase stays set until the softmax has consumed that tile.
-        const bool s_next = mbar_test(&s_full[(t + 1) % 3], ((t + 1) / 3) & 1);
-        // p = 2^(s * scale*log2e + bias - m_ref) in pairs; bf16 P for the MMA
-        float2 acc[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
-          const float2 pp = make_float2(ex2(x.x), ex2(x.y));   // MUFU; 2^-inf = +0 for masked columns
-          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pp);
-          pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
-        }
-        const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
-        const float2 a03 = fadd2(a01, a23);
-        l_run = l_run * alpha + (a03.x + a03.y);
-        m_run = m_new;
-        tmem_st16x2_32<32>(trow + buf * 128, pk);   // P keys 64h..64h+63 -> columns 32h..32h+31
-        if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
-          // rescale this half of the running output once P.V of the previous
-          // tile landed.  pv_done[u & 1] completes once per P.V of tile u, so
-          // P.V t-1 is phase (t-1)>>1 of pv_done[(t-1) & 1]; the phase before
-          // it (P.V t-3) has completed because S_t, ready here, was issued
-          // after P.V t-3, so the parity test is exact.
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, wc))) {
+          const int buf = t % 3;
+          if (!s_ready && !__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (t / 3) & 1, wc))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          bool need, s_next;
+          float alpha;
+          if (diag) {
+            constexpr int NC = R / 2;   // columns per thread: half of the row's own sub-block
+            uint32_t sr[NC];
+            if constexpr (NC == 32) {
+              tmem_ld16x2_sync1<32>(trow + buf * 128 + g_r * R, sr);
+            } else {
+              tmem_ld16x2_sync1_16<16>(trow + buf * 128 + g_r * R, sr);
+            }
+            float s[NC];
 #pragma unroll
-          for (int c0 = 0; c0 < DH; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld16x2_sync1<DH>(trow + kTmemO + c0, o);   // columns DH*h + c0..+31
+            for (int c = 0; c < NC; ++c) s[c] = __uint_as_float(sr[c]);
+            if (dcnt < R) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16x2_32<DH>(trow + kTmemO + c0, o);
+              for (int c = 0; c < NC; ++c) s[c] = (h * NC + c < dcnt) ? s[c] : -INFINITY;
+            }
+            float mxa[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxa[e] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < NC; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
+            const float mh = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+            const float mx = fmaxf(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 16)) * sl2;   // whole row
+            need = mx > m_run + kRescaleLog2;
+            const float m_new = need ? mx : m_run;
+            const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha = need ? ex2(m_run - m_ref) : 1.f;
+            const float neg = -m_ref;
+            s_next = mbar_test(&s_full[(t + 1) % 3], ((t + 1) / 3) & 1);
+            float2 acc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+            uint32_t pk[NC / 2];
+#pragma unroll
+            for (int c = 0; c < NC; c += 2) {
+              const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));   // MUFU: 2^-inf is +0 for masked columns
+              acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pp);
+              pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
+            }
+            const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+            const float2 a03 = fadd2(a01, a23);
+            l_run = l_run * alpha + (a03.x + a03.y);
+            m_run = m_new;
+            // P keys g_r*R + h*NC .. +NC-1 -> columns g_r*R/2 + h*NC/2 ..; zeros
+            // in the other sub-blocks' columns
+            const uint32_t zero[NC / 2] = {};
+            if constexpr (NC == 32) {
+              tmem_st16x2_16<16>(trow + buf * 128 + 32 * g_r, pk);
+              tmem_st16x2_16<16>(trow + buf * 128 + 32 * (1 - g_r), zero);
+            } else {
+              tmem_st16x2_8<8>(trow + buf * 128 + 16 * g_r, pk);
+#pragma unroll
+              for (int g2 = 1; g2 < 4; ++g2) tmem_st16x2_8<8>(trow + buf * 128 + 16 * ((g_r + g2) & 3), zero);
+            }
+          } else {
+            uint32_t sr[2][32];
+            // columns 64h + 0..31 and 64h + 32..63, waited for in the same statement
+            tmem_ld16x2_sync2<64>(trow + buf * 128, sr[0], trow + buf * 128 + 32, sr[1]);
+            float s[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+            if (cur.masked) {
+              const uint32_t w0 = h ? cur.mw[2] : cur.mw[0], w1 = h ? cur.mw[3] : cur.mw[1];
+#pragma unroll
+              for (int c = 0; c < 64; ++c) s[c] = ((((c < 32) ? w0 : w1) >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+              if (cur.pooled && (pb0 >= 0 || pb1 >= 0)) {
+                const int kk0 = (j - a.n_exact) * 128 + 64 * h;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) s[c] += (kk0 + c == pb0) ? d0 : ((kk0 + c == pb1) ? d1 : 0.f);
+              }
+            }
+            // half-row maximum: 8 independent chains of 3-input max
+            float mxa[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxa[e] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) mxa[(c >> 1) & 7] = fmax3(mxa[(c >> 1) & 7], s[c], s[c + 1]);
+            const float mh = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+            const float bias = cur.pooled ? log2b : 0.f;
+            const float mx = fmaxf(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 16)) * sl2 + bias;   // whole row
+            need = mx > m_run + kRescaleLog2;
+            const float m_new = need ? mx : m_run;
+            const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha = need ? ex2(m_run - m_ref) : 1.f;
+            const float neg = bias - m_ref;
+            // Is S of the next tile (t+1, possibly the next item's first) there
+            // already?  The test's latency overlaps the exponentials below, and a
+            // set phase stays set until the softmax has consumed that tile.
+            s_next = mbar_test(&s_full[(t + 1) % 3], ((t + 1) / 3) & 1);
+            // p = 2^(s * scale*log2e + bias - m_ref) in pairs; bf16 P for the MMA
+            float2 acc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float2 x = ffma2(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(neg, neg));
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));   // MUFU; 2^-inf = +0 for masked columns
+              acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pp);
+              pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
+            }
+            const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+            const float2 a03 = fadd2(a01, a23);
+            l_run = l_run * alpha + (a03.x + a03.y);
+            m_run = m_new;
+            tmem_st16x2_32<32>(trow + buf * 128, pk);   // P keys 64h..64h+63 -> columns 32h..32h+31
           }
+          if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+            // rescale this half of the running output once P.V of the previous
+            // tile landed.  pv_done[u & 1] completes once per P.V of tile u, so
+            // P.V t-1 is phase (t-1)>>1 of pv_done[(t-1) & 1]; the phase before
+            // it (P.V t-3) has completed because S_t, ready here, was issued
+            // after P.V t-3, so the parity test is exact.
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, wc))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < DH; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld16x2_sync1<DH>(trow + kTmemO + c0, o);   // columns DH*h + c0..+31
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16x2_32<DH>(trow + kTmemO + c0, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[buf]);
+          s_ready = __all_sync(0xFFFFFFFFu, s_next);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[buf]);
-        s_ready = __all_sync(0xFFFFFFFFu, s_next);
-      }
+      };
+      if (I.kind == 2) tile_loop(FlatTag<true>{}); else tile_loop(FlatTag<false>{});
       if (!ok) break;
       // epilogue: wait until every P.V of the item landed (a per-item barrier:
       // pv_done may still be two phases behind here, because the last tile's
