@@ -31,17 +31,21 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int it) {
     r.bh = it / a.q_tiles;
     r.slot0 = it % a.q_tiles;
     r.ntiles = (a.L + 127) / 128;
-  } else if (it < a.BH * a.items_sharp) {
-    r.kind = 1;
-    r.bh = it / a.items_sharp;
-    r.slot0 = (it % a.items_sharp) * G;
-    r.ntiles = (a.T_kv + G - 1) / G;
   } else {
-    it -= a.BH * a.items_sharp;
-    r.kind = 2;
-    r.bh = it / a.items_flat;
-    r.slot0 = (it % a.items_flat) * G;
-    r.ntiles = a.n_exact + (a.T_kv + 127) / 128;
+    // head by head: a head's sharp items, then its flat items, so the flat
+    // items' exact blocks are read while the head's kept K/V is still in L2
+    const int per_head = a.items_sharp + a.items_flat;
+    r.bh = it / per_head;
+    const int k = it % per_head;
+    if (k < a.items_sharp) {
+      r.kind = 1;
+      r.slot0 = k * G;
+      r.ntiles = (a.T_kv + G - 1) / G;
+    } else {
+      r.kind = 2;
+      r.slot0 = (k - a.items_sharp) * G;
+      r.ntiles = a.n_exact + (a.T_kv + 127) / 128;
+    }
   }
   return r;
 }
