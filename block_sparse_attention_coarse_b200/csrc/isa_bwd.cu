@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(128) bwd_zero_unkept_kernel(const int* __restr
 // key/value-stationary kernel: dK, dV
 // ---------------------------------------------------------------------------
 // An item is one 128-row key/value tile of one head and stays in shared
-// memory while 64-row query steps stream past it:
+// memory while 128-row query steps stream past it:
 //   kept launch   : rows = G = 128/R consecutive kept blocks (kept positions
 //                   tile*G ..); steps = every sharp block, then the flat
 //                   blocks whose exact list holds one of the tile's blocks
@@ -122,61 +122,68 @@ __global__ void __launch_bounds__(128) bwd_zero_unkept_kernel(const int* __restr
 //   pooled launch : rows = 128 consecutive pooled kept blocks (Kp/Vp rows);
 //                   steps = every flat block, with the flat block's own exact
 //                   blocks masked out; log-weight log2(n_j) per row
-// Per step (TMEM lane = key/value row):
-//   S^T = K Q^T, dP^T = V dO^T         (SS, M=128, N=64, K=D)
-//   P^T = 2^(S^T s log2e + w_j - lse2), dS^T = P^T (dP^T - Delta)   (softmax warps)
+// A step is GQ = 128/R query blocks (128 query columns).  Per step u (TMEM
+// lane = key/value row):
+//   S^T = K Q^T, dP^T = V dO^T         (SS, M=128, N=128, K=D)
+//   P^T = 2^(S^T s log2e + w_j - lse2)                      (softmax, phase A)
+//   dS^T = P^T (dP^T - Delta)                               (softmax, phase B)
 //   dV += P^T dO, dK += dS^T Q         (TS: P^T / dS^T read as bf16 from TMEM)
+// The tensor core runs 128 x 128 k-steps at full rate only from N = 128 up
+// (N = 64 takes as long as N = 128), so steps are 128 query rows wide, and
+// TMEM then holds one S^T and one dP^T buffer beside dV and dK.  The four
+// products of consecutive steps are issued as dV_u, S^T_{u+1}, dK_u,
+// dP^T_{u+1}: phase A of step u+1 (the exponentials) runs behind dK_u and
+// dP^T_{u+1}, phase B behind dV_{u+1} and S^T_{u+2}.  A product that
+// overwrites a buffer is issued after the one that reads it; the tensor
+// pipe runs one thread's MMAs in order.
 // Roles (576 threads, one CTA per SM): warp 0 producer (the whole warp finds
 // the steps; lane 0 loads the tile, publishes each step's metadata and
 // issues its copies), warp 1 MMA issuer (converged, one elected lane),
-// warps 2..17: warp w owns TMEM lanes 32*(w%4).. and query
-// columns 16*((w-2)/4).. of each step (four warps per lane quarter, so that
-// each scheduler interleaves four of them), and writes the epilogue.
+// warps 2..17: warp w owns TMEM lanes 32*(w%4).. and query columns
+// 32*((w-2)/4).. of each step (four warps per lane quarter, so that each
+// scheduler interleaves four of them), and writes the epilogue.
 constexpr int kKvSoft = 16;                      // softmax warps
 constexpr int kKvThreads = 64 + 32 * kKvSoft;
-constexpr int kNSQ = 3;           // query/dO step stages
-// TMEM: S^T and dP^T of two steps (step u in buffer u % 2, so the next
-// step's products run while the softmax warps work on this one); each
-// softmax warp packs its bf16 P^T / dS^T into the first half of the 16
-// fp32 columns it has just read, where the dV / dK products take them as
-// the A operand; then dV and dK.
-constexpr uint32_t kTST = 0;      // S^T then P^T, two buffers of 64 columns
-constexpr uint32_t kTDP = 128;    // dP^T then dS^T, two buffers of 64 columns    // two buffers of 64 columns: P^T (bf16 pairs) at +0, dS^T at +32
+constexpr int kNSQ = 2;           // query/dO step stages
+// TMEM: S^T then P^T, dP^T then dS^T (each softmax warp packs its bf16
+// values of query columns 16k..16k+15 into columns 16k..16k+7 of the fp32
+// columns it has just read, where the dV / dK products take them as the A
+// operand); then dV and dK.
+constexpr uint32_t kTST = 0;      // S^T, then P^T
+constexpr uint32_t kTDP = 128;    // dP^T, then dS^T
 constexpr uint32_t kTDV = 256;    // dV accumulator (D columns); dK at kTDV + D
 
 template <int D, int R>
 struct KvCfg {
   static constexpr int G = 128 / R;               // kept blocks per tile
-  static constexpr int GQ = 64 / R;               // query blocks per step
+  static constexpr int GQ = 128 / R;              // query blocks per step
   static constexpr int NCH = D / 64;              // 64-column chunks of a row
   static constexpr uint32_t CHUNK = 128 * 128;    // 128 rows x 128 bytes
-  static constexpr uint32_t QCHUNK = 64 * 128;    // 64 rows x 128 bytes
-  static constexpr uint32_t TILE = 128 * D * 2;
-  static constexpr uint32_t QTILE = 64 * D * 2;
+  static constexpr uint32_t TILE = 128 * D * 2;   // one 128-row tile (K, V, a Q or a dO step)
   static constexpr uint32_t BOX = R * 128;        // one TMA box
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = TILE;
   static constexpr uint32_t Q_OFF = 2 * TILE;
-  static constexpr uint32_t DO_OFF = Q_OFF + kNSQ * QTILE;
-  static constexpr uint32_t DL_OFF = DO_OFF + kNSQ * QTILE;   // (lse2, Delta) of the 64 step rows
-  static constexpr uint32_t DL_STAGE = 64 * 8;
+  static constexpr uint32_t DO_OFF = Q_OFF + kNSQ * TILE;
+  static constexpr uint32_t DL_OFF = DO_OFF + kNSQ * TILE;   // (lse2, Delta) of the 128 step rows
+  static constexpr uint32_t DL_STAGE = 128 * 8;
   static constexpr uint32_t SMEM_USED = DL_OFF + kNSQ * DL_STAGE + 1024;
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits on an SM
   static constexpr uint32_t SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static constexpr uint32_t ID_T = idesc_bf16_f32(128, 64, 0);
+  static constexpr uint32_t ID_T = idesc_bf16_f32(128, 128, 0);
   static constexpr uint32_t ID_A = idesc_bf16_f32(128, D, 1);
 };
 
 struct StepMeta {
-  int blk[2];             // block ids of the step's query blocks
-  int start[2], cnt[2];   // token start and valid rows of the step's query blocks
-  uint32_t m[2][4];       // tile rows each query block attends (bit r of m[g][r/32])
+  int blk[4];             // block ids of the step's query blocks
+  int start[4], cnt[4];   // token start and valid rows of the step's query blocks
+  uint32_t m[4][4];       // tile rows each query block attends (bit r of m[g][r/32])
   int last;               // last step of the item
 };
 
 __device__ __forceinline__ void clear_meta(StepMeta& m) {
 #pragma unroll
-  for (int g = 0; g < 2; ++g) {
+  for (int g = 0; g < 4; ++g) {
     m.blk[g] = 0;
     m.start[g] = 0;
     m.cnt[g] = 0;
@@ -194,9 +201,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                   const BwdArgs b) {
   using C = KvCfg<D, R>;
   constexpr int G = C::G, GQ = C::GQ;
+  static_assert(GQ <= 4, "StepMeta holds four query blocks");
   const AttnArgs& a = b.a;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t kv_full, kv_empty, q_full[kNSQ], q_empty[kNSQ], sd_full[2], ds_full[2];
+  __shared__ __align__(8) uint64_t kv_full, kv_empty, q_full[kNSQ], q_empty[kNSQ];
+  __shared__ __align__(8) uint64_t s_full, dp_full, p_ready, ds_ready;
   __shared__ __align__(8) uint64_t acc_ready, acc_free, drain_bar, inject_bar;
   __shared__ StepMeta meta[kNSQ];
   __shared__ uint32_t tmem_base_sh;
@@ -214,11 +223,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    mbar_init(&sd_full[0], 1);
-    mbar_init(&sd_full[1], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&ds_full[i], 32 * kKvSoft);
+    mbar_init(&s_full, 1);
+    mbar_init(&dp_full, 1);
+    mbar_init(&p_ready, kKvSoft);    // one arrival per softmax warp
+    mbar_init(&ds_ready, kKvSoft);
     mbar_init(&acc_ready, 1);
-    mbar_init(&acc_free, 32 * kKvSoft);
+    mbar_init(&acc_free, kKvSoft);
     mbar_init(&drain_bar, 1);
     mbar_init(&inject_bar, 1);
     abort_flag = 0;
@@ -283,15 +293,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (u >= kNSQ && !mbar_wait(&q_empty[s], ((u / kNSQ) - 1) & 1, wc)) return false;
         meta[s] = m;
         meta[s].last = last;   // published by the arrive below (release), read after q_full (acquire)
-        mbar_arrive_expect_tx(&q_full[s], 2 * C::QTILE + C::DL_STAGE);
+        mbar_arrive_expect_tx(&q_full[s], 2 * C::TILE + C::DL_STAGE);
         ++qcnt[s];
         for (int g = 0; g < GQ; ++g) {
           const int row = bh * a.L + (m.cnt[g] > 0 ? m.start[g] : 0);
           bulk_load_1d(sgen + C::DL_OFF + s * C::DL_STAGE + g * R * 8,
                        b.dl + ((size_t)bh * (a.T_src + a.T_ctx) + m.blk[g]) * R, R * 8, &q_full[s]);
           for (int c = 0; c < C::NCH; ++c) {
-            tma_load_2d(sgen + C::Q_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[s]);
-            tma_load_2d(sgen + C::DO_OFF + s * C::QTILE + c * C::QCHUNK + g * C::BOX, &tm_do, c * 64, row,
+            tma_load_2d(sgen + C::Q_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[s]);
+            tma_load_2d(sgen + C::DO_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, &tm_do, c * 64, row,
                         &q_full[s]);
           }
         }
@@ -390,65 +400,74 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per step u: dV_u (needs P^T_u), S^T_{u+1} (overwrites P^T_u), dK_u
+    // (needs dS^T_u), dP^T_{u+1} (overwrites dS^T_u).  One commit per product
+    // group that someone waits for.
     bool issued = false, ok = true;
     if (a.inject) ok = warp_wait(&inject_bar, 0, wc);   // nothing arrives: runs out
     int u = 0, n = 0;
     const uint64_t kdesc = smem_desc_sw128(sbase + C::K_OFF, 16, 1024);
     const uint64_t vdesc = smem_desc_sw128(sbase + C::V_OFF, 16, 1024);
-    // S^T and dP^T of step uu into buffer uu % 2
-    auto issue_t = [&](int uu) -> bool {
+    // S^T of step uu (waits for its query/dO stage)
+    auto issue_s = [&](int uu) -> bool {
       const int s = uu % kNSQ;
-      if (!warp_wait(&q_full[s], (uu / kNSQ) & 1, wc))
-        return false;
+      if (!warp_wait(&q_full[s], (uu / kNSQ) & 1, wc)) return false;
       tc_fence_after();
-      const uint64_t qd = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, 16, 1024);
-      const uint64_t dd = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, 16, 1024);
+      const uint64_t qd = smem_desc_sw128(sbase + C::Q_OFF + s * C::TILE, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
-        const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
-        mma_ss_elect(tmem + kTST + (uu & 1) * 64, kdesc + oa, qd + ob, C::ID_T, ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t oa = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
-        const uint32_t ob = ((ks >> 2) * C::QCHUNK + (ks & 3) * 32) >> 4;
-        mma_ss_elect(tmem + kTDP + (uu & 1) * 64, vdesc + oa, dd + ob, C::ID_T, ks > 0);
+        const uint32_t o = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTST, kdesc + o, qd + o, C::ID_T, ks > 0);
       }
       issued = true;
-      tc_commit_elect(&sd_full[uu & 1]);
+      tc_commit_elect(&s_full);
       return true;
+    };
+    // dP^T of step uu (its stage already waited for by issue_s)
+    auto issue_dp = [&](int uu) {
+      const int s = uu % kNSQ;
+      const uint64_t dd = smem_desc_sw128(sbase + C::DO_OFF + s * C::TILE, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = ((ks >> 2) * C::CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss_elect(tmem + kTDP, vdesc + o, dd + o, C::ID_T, ks > 0);
+      }
+      tc_commit_elect(&dp_full);
     };
     for (int it = blockIdx.x; ok && it < b.kv_total; it += gridDim.x, ++n) {
       if (!warp_wait(&kv_full, n & 1, wc)) break;
       tc_fence_after();
-      if (!(ok = issue_t(u))) break;
+      if (!(ok = issue_s(u))) break;
+      issue_dp(u);
       for (bool first = true;; first = false) {
         const int s = u % kNSQ;
-        const int last = meta[s].last;
-        // the next step's S^T, dP^T go to the other buffers while the softmax
-        // warps work on this one
-        if (!last && !(ok = issue_t(u + 1))) break;
-        if (!warp_wait(&ds_full[u & 1], (u >> 1) & 1, wc) ||
-            (first && n > 0 && !warp_wait(&acc_free, (n - 1) & 1, wc))) {
+        const int last = meta[s].last;   // read after q_full[s] (issue_s)
+        const uint64_t qmn = smem_desc_sw128(sbase + C::Q_OFF + s * C::TILE, C::CHUNK, 1024);
+        const uint64_t dmn = smem_desc_sw128(sbase + C::DO_OFF + s * C::TILE, C::CHUNK, 1024);
+        // dV += P^T dO: packed P^T of query columns 16k..16k+15 (one K step)
+        // sits in columns 16k..16k+7
+        if (!warp_wait(&p_ready, u & 1, wc) || (first && n > 0 && !warp_wait(&acc_free, (n - 1) & 1, wc))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t qmn = smem_desc_sw128(sbase + C::Q_OFF + s * C::QTILE, C::QCHUNK, 1024);
-        const uint64_t dmn = smem_desc_sw128(sbase + C::DO_OFF + s * C::QTILE, C::QCHUNK, 1024);
-        const uint32_t pk = (u & 1) * 64;
-        // packed bf16 P^T / dS^T: query columns 16q..16q+15 (one K step) sit
-        // in the buffer's columns 16q..16q+7
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ts_elect(tmem + kTDV, tmem + kTST + pk + ks * 16, dmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_elect(tmem + kTDV, tmem + kTST + ks * 16, dmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
                        (!first || ks > 0) ? 1u : 0u);
+        if (!last && !(ok = issue_s(u + 1))) break;
+        // dK += dS^T Q
+        if (!warp_wait(&ds_ready, u & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ts_elect(tmem + kTDV + D, tmem + kTDP + pk + ks * 16, qmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_elect(tmem + kTDV + D, tmem + kTDP + ks * 16, qmn + (uint64_t)(ks * 2048 >> 4), C::ID_A,
                        (!first || ks > 0) ? 1u : 0u);
-        tc_commit_elect(&q_empty[s]);
+        tc_commit_elect(&q_empty[s]);   // last reads of Q_u and dO_u
+        if (!last) issue_dp(u + 1);
         ++u;
         if (last) break;
       }
@@ -465,8 +484,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int quarter = warp & 3, qd = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                      // tile row = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int gq = (R == 32) ? (qd >> 1) : 0;               // this thread's query block of a step
-    const int coff = (R == 32) ? 16 * (qd & 1) : 16 * qd;   // its first column within that block
+    const int c0 = 32 * qd;                                 // this warp's first query column of a step
+    const int gq = c0 / R;                                  // the query block of its 32 columns
     const float sl2 = a.sl2;
     constexpr int DQ = D / 4;                               // epilogue columns of dV and of dK
     int u = 0, n = 0;
@@ -493,42 +512,76 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
       }
       for (;;) {
-        const int s = u % kNSQ, buf = u & 1;
-        // sd_full follows q_full of the same step (the MMAs waited for it);
+        const int s = u % kNSQ;
+        // s_full follows q_full of the same step (the MMAs waited for it);
         // the q_full test makes the bulk-copied (lse2, Delta) visible here
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sd_full[buf], (u >> 1) & 1, wc) &&
-                                         mbar_wait(&q_full[s], (u / kNSQ) & 1, wc))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full, u & 1, wc) && mbar_wait(&q_full[s], (u / kNSQ) & 1, wc))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const int last = meta[s].last;
         const bool on = row_valid && ((meta[s].m[gq][r >> 5] >> (r & 31)) & 1u);
-        // (lse2, Delta) of this thread's 16 columns, two columns per 16-byte
+        // (lse2, Delta) of this warp's 32 columns, two columns per 16-byte
         // broadcast load; rows past a block's end hold (inf, 0), so P = 0 there
-        const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE) + (gq * R + coff) / 2;
-        float4 ld[8];
+        const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE) + c0 / 2;
+        // phase A: P^T, 16 columns at a time
+        float p[32];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ld[e] = dls[e];
-        uint32_t sv[16], dp[16];
-        tmem_ld16_pair_sync(tl + kTST + buf * 64 + 16 * qd, sv, tl + kTDP + buf * 64 + 16 * qd, dp);
-        uint32_t pp[8], pd[8];
+        for (int h = 0; h < 2; ++h) {
+          float2 lz[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float4 x = ld[e >> 1];
-          float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, bias - x.x));
-          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, bias - x.z));
-          if (!on) p0 = p1 = 0.f;
-          const float g0 = p0 * (__uint_as_float(dp[e]) - x.y);
-          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - x.w);
-          pp[e >> 1] = pack_bf16x2(p0, p1);
-          pd[e >> 1] = pack_bf16x2(g0, g1);
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = dls[8 * h + e];
+            lz[e] = make_float2(bias - x.x, bias - x.z);
+          }
+          uint32_t sv[16];
+          tmem_ld16_sync(tl + kTST + c0 + 16 * h, sv);
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, lz[e >> 1].x));
+            float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, lz[e >> 1].y));
+            if (!on) p0 = p1 = 0.f;
+            p[16 * h + e] = p0;
+            p[16 * h + e + 1] = p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st8(tl + kTST + c0 + 16 * h, pk);
         }
-        tmem_st8(tl + kTST + buf * 64 + 16 * qd, pp);
-        tmem_st8(tl + kTDP + buf * 64 + 16 * qd, pd);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ds_full[buf]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready);
+        // phase B: dS^T = P^T (dP^T - Delta)
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&dp_full, u & 1, wc))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float2 dz[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = dls[8 * h + e];
+            dz[e] = make_float2(x.y, x.w);
+          }
+          uint32_t dp[16];
+          tmem_ld16_sync(tl + kTDP + c0 + 16 * h, dp);
+          uint32_t pd[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const float g0 = p[16 * h + e] * (__uint_as_float(dp[e]) - dz[e >> 1].x);
+            const float g1 = p[16 * h + e + 1] * (__uint_as_float(dp[e + 1]) - dz[e >> 1].y);
+            pd[e >> 1] = pack_bf16x2(g0, g1);
+          }
+          tmem_st8(tl + kTDP + c0 + 16 * h, pd);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_ready);
         ++u;
         if (last) break;
       }
@@ -551,7 +604,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         if (part == 1) {
           tc_fence_before();
-          mbar_arrive(&acc_free);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_free);
         }
         if (!row_valid) continue;
         const float f = part ? sc : 1.f;
@@ -574,11 +628,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) x[i] = f * __uint_as_float(g[(e + i) >> 4][(e + i) & 15]);
             if (b.has_pooled) {
-              const float4 c0 = pc[e >> 2], c1 = pc[(e >> 2) + 1];
-              x[0] = fmaf(c0.x, inv, x[0]); x[1] = fmaf(c0.y, inv, x[1]);
-              x[2] = fmaf(c0.z, inv, x[2]); x[3] = fmaf(c0.w, inv, x[3]);
-              x[4] = fmaf(c1.x, inv, x[4]); x[5] = fmaf(c1.y, inv, x[5]);
-              x[6] = fmaf(c1.z, inv, x[6]); x[7] = fmaf(c1.w, inv, x[7]);
+              const float4 c0v = pc[e >> 2], c1v = pc[(e >> 2) + 1];
+              x[0] = fmaf(c0v.x, inv, x[0]); x[1] = fmaf(c0v.y, inv, x[1]);
+              x[2] = fmaf(c0v.z, inv, x[2]); x[3] = fmaf(c0v.w, inv, x[3]);
+              x[4] = fmaf(c1v.x, inv, x[4]); x[5] = fmaf(c1v.y, inv, x[5]);
+              x[6] = fmaf(c1v.z, inv, x[6]); x[7] = fmaf(c1v.w, inv, x[7]);
             }
             dst[e >> 3] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                                      pack_bf16x2(x[6], x[7]));
