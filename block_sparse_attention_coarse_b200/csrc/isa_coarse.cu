@@ -10,118 +10,209 @@
 // added as gamma * O_coarse_i to every token of query block i; gamma is the
 // caller's scalar.
 //
-// The work is T x T x D per head (a few GFLOP at 32K tokens), so these are
-// CUDA-core kernels, one CTA per (head, block), 256 threads:
-//   coarse_fwd_kernel   scores of up to 8 query blocks against all T pooled keys
-//                       (one key per thread), softmax, O_coarse, and the
-//                       read-modify-write of the blocks' output rows
-//   coarse_bwd_q_kernel per query block i: dO_i = gamma * sum of the block's
-//                       dout rows, Delta_i = dO_i . O_i, dS_ij =
-//                       P_ij (dO_i . Vc_j - Delta_i), dQc_i = s sum_j dS_ij Kc_j
-//                       -> dq rows += dQc_i / n_i; keeps (lse2_i, Delta_i) and
-//                       dO_i for the key pass; dgamma partial
+// The work is dense attention over the T pooled blocks of a head (T x T x D),
+// kept in fp32 on the CUDA cores: the pooled means are fp32, and a bf16
+// tensor-core product would round the logits far beyond the residual's
+// tolerance.  Each CTA (256 threads) takes 64 query (or key) blocks and walks
+// the other side in tiles of 64 rows staged in shared memory; a thread owns a
+// 4 x 4 micro-tile of each 64 x 64 score tile (rows 4 ty .. 4 ty + 3, columns
+// tx, tx + 16, tx + 32, tx + 48) and 4 rows x D/16 columns of each 64 x D
+// product; softmax rows run online (running maximum and sum), as in flash
+// attention:
+//   coarse_fwd_kernel    O_coarse of 64 query blocks -> out rows += gamma O_i
+//   coarse_bwd_q_kernel  per query block i: the forward again (lse2_i, O_i),
+//                        dO_i = gamma * sum of the block's dout rows, Delta_i =
+//                        dO_i . O_i, dgamma += (dout sum) . O_i; then dS_ij =
+//                        P_ij (dO_i . Vc_j - Delta_i), dQc_i = s sum_j dS_ij Kc_j
+//                        -> dq rows += dQc_i / n_i; keeps (lse2_i, Delta_i) and
+//                        dO_i for the key pass
 //   coarse_bwd_kv_kernel per key block j: dKc_j = s sum_i dS_ij Qc_i,
-//                       dVc_j = sum_i P_ij dO_i -> dk, dv rows += (.) / n_j
+//                        dVc_j = sum_i P_ij dO_i -> dk, dv rows += (.) / n_j
 // Gradients reach the tokens through the pooled means (Kc_j is the mean of
 // block j's n_j keys), as in the sparse path's backward.
-#include <algorithm>
-
 #include "isa_common.cuh"
 
 namespace isa {
 namespace coarse {
 
 constexpr int kThreads = 256;
+constexpr int kBM = 64;   // blocks per CTA and per tile
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr int kRows = 8;           // most query (key) blocks per CTA
+template <int D>
+struct Tile {
+  static constexpr int LD = D + 4;              // row stride (floats) of a 64 x D operand tile
+  static constexpr int LP = kBM + 4;            // row stride of a 64 x 64 weight tile
+  static constexpr int OP = kBM * LD;           // floats of an operand tile
+  static constexpr int WP = kBM * LP;           // floats of a weight tile
+  static constexpr int NC = D / 16;             // product columns per thread
+};
 
-// Softmax of rows r < nr of pr[r * ld .. + T) in place (log2-unit scores),
-// one warp per row; lse2[r] receives each row's log2 normaliser.
-__device__ void rows_softmax(float* pr, int ld, int T, int nr, float* lse2) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp < nr) {
-    float* row = pr + (size_t)warp * ld;
-    float m = -INFINITY;
-    for (int j = lane; j < T; j += 32) m = fmaxf(m, row[j]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-    float l = 0.f;
-    for (int j = lane; j < T; j += 32) {
-      const float e = exp2f(row[j] - m);
-      row[j] = e;
-      l += e;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-    const float inv = 1.f / l;
-    for (int j = lane; j < T; j += 32) row[j] *= inv;
-    if (lane == 0) lse2[warp] = m + __log2f(l);
+struct CoarseArgs {
+  const float *Qc, *Kc, *Vc;   // plan: [BH, T, D]
+  int T, T_src, L, L_src, L_ctx, b;
+  float sl2, scale, gamma;
+  __nv_bfloat16* out;          // forward: out += gamma * O_coarse
+  const __nv_bfloat16* dout;   // backward
+  __nv_bfloat16 *dq, *dk, *dv;
+  float* dgamma;               // [BH] or null
+  float2* stat;                // [BH, T] (lse2_i, Delta_i)
+  float* dO;                   // [BH, T, D] gamma * block sums of dout
+};
+
+// Xs (64 x LD) = rows [r0, r0 + 64) of X (fp32 [n, D]), zero past n.
+template <int D>
+__device__ void load_tile(float* Xs, const float* __restrict__ X, int r0, int n) {
+  constexpr int V4 = D / 4;
+  for (int e = threadIdx.x; e < kBM * V4; e += kThreads) {
+    const int r = e / V4, c4 = e % V4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < n) v = *reinterpret_cast<const float4*>(X + (size_t)(r0 + r) * D + 4 * c4);
+    *reinterpret_cast<float4*>(Xs + r * Tile<D>::LD + 4 * c4) = v;
   }
-  __syncthreads();
 }
 
-// out[r][d] = sum_j w[r * ld + j] X[j][d] for r < nr (shared out [kRows][D]):
-// each thread owns one column and a contiguous slice of j, with kRows
-// accumulators, so every X row is read once for all nr rows, and the
-// weights of 4 consecutive j come in one 16-byte broadcast load (ld is a
-// multiple of 4 and w is zero in [T, ld)); slices combined through `part`.
+// acc[a][c] = A[4 ty + a] . B[tx + 16 c] over D (A, B: 64 x LD tiles)
 template <int D>
-__device__ void rows_combine(const float* w, int ld, int nr, const float* __restrict__ X, int T, float* out,
-                             float* part) {
-  constexpr int SPLIT = kThreads / D;
-  const int d = threadIdx.x % D, h = threadIdx.x / D;
-  const int chunk = ((ld / 4 + SPLIT - 1) / SPLIT) * 4;
-  const int j0 = h * chunk, j1 = min(j0 + chunk, ld);
-  float acc[kRows];
+__device__ __forceinline__ void tile_dots(const float* A, const float* B, float (&acc)[4][4]) {
+  constexpr int LD = Tile<D>::LD;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
-  for (int j = j0; j < j1; j += 4) {
-    float x[4];
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = (j + i < T) ? X[(size_t)(j + i) * D + d] : 0.f;
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      if (r < nr) {
-        const float4 wv = *reinterpret_cast<const float4*>(w + (size_t)r * ld + j);
-        acc[r] = fmaf(wv.x, x[0], fmaf(wv.y, x[1], fmaf(wv.z, x[2], fmaf(wv.w, x[3], acc[r]))));
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) part[(h * kRows + r) * D + d] = acc[r];
-  __syncthreads();
-  for (int e = threadIdx.x; e < nr * D; e += kThreads) {
-    const int r = e / D, c = e % D;
-    float sum = 0.f;
-    for (int k = 0; k < SPLIT; ++k) sum += part[(k * kRows + r) * D + c];
-    out[r * D + c] = sum;
-  }
-  __syncthreads();
-}
-
-// acc[r] = A[r] . x for r < nr: the rows of A in shared memory (read as
-// 16-byte broadcasts: every lane of a warp reads the same address), x one
-// row of global memory per thread.  Threads take different x rows, so no
-// shuffle reduction is needed.
-template <int D>
-__device__ __forceinline__ void row_dots(const float* A, int nr, const float* __restrict__ x, float (&acc)[kRows]) {
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
 #pragma unroll 4
-  for (int c = 0; c < D; c += 4) {
-    const float4 xv = *reinterpret_cast<const float4*>(x + c);
+  for (int d = 0; d < D; d += 4) {
+    float4 qa[4], kb[4];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      if (r < nr) {
-        const float4 av = *reinterpret_cast<const float4*>(A + r * D + c);
-        acc[r] = fmaf(av.x, xv.x, fmaf(av.y, xv.y, fmaf(av.z, xv.z, fmaf(av.w, xv.w, acc[r]))));
+    for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const float4*>(A + (4 * ty + a) * LD + d);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) kb[c] = *reinterpret_cast<const float4*>(B + (tx + 16 * c) * LD + d);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[a][c] = fmaf(qa[a].x, kb[c].x, acc[a][c]);
+        acc[a][c] = fmaf(qa[a].y, kb[c].y, acc[a][c]);
+        acc[a][c] = fmaf(qa[a].z, kb[c].z, acc[a][c]);
+        acc[a][c] = fmaf(qa[a].w, kb[c].w, acc[a][c]);
+      }
+  }
+}
+
+// acc[a][n] += sum_k W[4 ty + a][k] X[k][col n]: W a 64 x LP weight tile, X a
+// 64 x LD operand tile; this thread's columns are 4 tx + 64 g + (0..3)
+template <int D>
+__device__ __forceinline__ void tile_mul(const float* W, const float* X, float (&acc)[4][Tile<D>::NC]) {
+  constexpr int LD = Tile<D>::LD, LP = Tile<D>::LP, NG = D / 64;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll 2
+  for (int k = 0; k < kBM; k += 4) {
+    float4 w[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) w[a] = *reinterpret_cast<const float4*>(W + (4 * ty + a) * LP + k);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const float4 x = *reinterpret_cast<const float4*>(X + (k + kk) * LD + 4 * tx + 64 * g);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float wv = kk == 0 ? w[a].x : kk == 1 ? w[a].y : kk == 2 ? w[a].z : w[a].w;
+          acc[a][4 * g + 0] = fmaf(wv, x.x, acc[a][4 * g + 0]);
+          acc[a][4 * g + 1] = fmaf(wv, x.y, acc[a][4 * g + 1]);
+          acc[a][4 * g + 2] = fmaf(wv, x.z, acc[a][4 * g + 2]);
+          acc[a][4 * g + 3] = fmaf(wv, x.w, acc[a][4 * g + 3]);
+        }
       }
     }
   }
 }
 
-// rows [t0, t0+n) of x (bf16 [.., D]) += scale * v (shared fp32 [D])
+// W[4 ty + a][tx + 16 c] = v[a][c]
+template <int D>
+__device__ __forceinline__ void store_weights(float* W, const float (&v)[4][4]) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) W[(4 * ty + a) * Tile<D>::LP + tx + 16 * c] = v[a][c];
+}
+
+// x over the 16 threads of a micro-tile row (lanes 16 (ty & 1) + tx)
+__device__ __forceinline__ float row_max16(float x) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+  return x;
+}
+__device__ __forceinline__ float row_sum16(float x) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+// The forward of this CTA's 64 query rows (Qs) over all T keys: running
+// maximum m and sum l (log2 units) per row and the unnormalised O.  Uses Ks
+// (then the weight tile) and Vs as scratch.
+template <int D>
+__device__ void flash_rows(const CoarseArgs& a, size_t hb, const float* Qs, float* Ks, float* Vs, float (&m)[4],
+                           float (&l)[4], float (&O)[4][Tile<D>::NC]) {
+  const int tx = threadIdx.x & 15;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.f;
+#pragma unroll
+    for (int n = 0; n < Tile<D>::NC; ++n) O[r][n] = 0.f;
+  }
+  for (int j0 = 0; j0 < a.T; j0 += kBM) {
+    __syncthreads();   // the previous tile's readers are done
+    load_tile<D>(Ks, a.Kc + hb, j0, a.T);
+    load_tile<D>(Vs, a.Vc + hb, j0, a.T);
+    __syncthreads();
+    float s[4][4];
+    tile_dots<D>(Qs, Ks, s);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float cm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[r][c] = (j0 + tx + 16 * c < a.T) ? s[r][c] * a.sl2 : -INFINITY;
+        cm = fmaxf(cm, s[r][c]);
+      }
+      const float mn = fmaxf(m[r], row_max16(cm));   // finite: key j0 + 0 < T
+      const float alpha = exp2f(m[r] - mn);           // 0 on the first tile
+      float ps = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[r][c] = exp2f(s[r][c] - mn);
+        ps += s[r][c];
+      }
+      l[r] = l[r] * alpha + row_sum16(ps);
+      m[r] = mn;
+#pragma unroll
+      for (int n = 0; n < Tile<D>::NC; ++n) O[r][n] *= alpha;
+    }
+    __syncthreads();   // every thread has read Ks: the weights take its place
+    store_weights<D>(Ks, s);
+    __syncthreads();
+    tile_mul<D>(Ks, Vs, O);
+  }
+}
+
+// Xs (64 x LD) = the thread's 4 x NC values (rows 4 ty + r, columns 4 tx + 64 g + i)
+template <int D>
+__device__ __forceinline__ void stage_rows(float* Xs, const float (&v)[4][Tile<D>::NC]) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int g = 0; g < D / 64; ++g)
+      *reinterpret_cast<float4*>(Xs + (4 * ty + r) * Tile<D>::LD + 4 * tx + 64 * g) =
+          make_float4(v[r][4 * g], v[r][4 * g + 1], v[r][4 * g + 2], v[r][4 * g + 3]);
+}
+
+// rows [t0, t0 + n) of x (bf16 [.., D]) += scale * v (fp32 [D] in shared memory)
 template <int D>
 __device__ void add_rows(__nv_bfloat16* x, size_t t0, int n, const float* v, float scale) {
   for (int e = threadIdx.x; e < n * (D / 8); e += kThreads) {
@@ -138,222 +229,222 @@ __device__ void add_rows(__nv_bfloat16* x, size_t t0, int n, const float* v, flo
   }
 }
 
-struct CoarseArgs {
-  const float *Qc, *Kc, *Vc;   // plan: [BH, T, D]
-  int T, T_src, L, L_src, L_ctx, b;
-  int rows;                    // query (key) blocks per CTA, <= kRows
-  float sl2, scale, gamma;
-  __nv_bfloat16* out;          // forward: out += gamma * O_coarse
-  const __nv_bfloat16* dout;   // backward
-  __nv_bfloat16 *dq, *dk, *dv;
-  float* dgamma;               // [BH] or null
-  float2* stat;                // [BH, T] (lse2_i, Delta_i)
-  float* dO;                   // [BH, T, D] gamma * block sums of dout
-};
-
-// Shared memory: D-vectors first (read as float4 / float2), then the
-// combine scratch, then the [rows][T] score rows.
-template <int D>
-constexpr int kVecFloats = 2 * kRows * D;
-template <int D>
-constexpr int kPartFloats = (kThreads / D) * kRows * D;
-
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_fwd_kernel(const CoarseArgs a) {
+  using C = Tile<D>;
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                          // [kRows][D] Qc rows
-  float* oc = qs + kRows * D;              // [kRows][D] O_coarse rows
-  float* part = oc + kRows * D;            // combine scratch
-  float* lse2 = part + kPartFloats<D>;     // [kRows]
-  float* pr = lse2 + kRows;                // [rows][ld], zero past T
-  const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
-  const int nr = min(a.rows, a.T - i0);
-  const int ld = (a.T + 3) & ~3;
+  float* Qs = sm;
+  float* Ks = Qs + C::OP;   // K tile, then the weights; finally O_coarse rows
+  float* Vs = Ks + C::OP;
+  const int bh = blockIdx.y, i0 = blockIdx.x * kBM;
+  const int nr = min(kBM, a.T - i0);
   const size_t hb = (size_t)bh * a.T * D;
-  for (int e = threadIdx.x; e < nr * D; e += kThreads) qs[e] = a.Qc[hb + (size_t)i0 * D + e];
-  __syncthreads();
-  // scores: one key block per thread, against all nr query rows
-  for (int j = threadIdx.x; j < ld; j += kThreads) {
-    float acc[kRows];
-    if (j < a.T) row_dots<D>(qs, nr, a.Kc + hb + (size_t)j * D, acc);
+  load_tile<D>(Qs, a.Qc + hb, i0, a.T);
+  float m[4], l[4], O[4][C::NC];
+  flash_rows<D>(a, hb, Qs, Ks, Vs, m, l, O);
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < nr) pr[(size_t)r * ld + j] = j < a.T ? acc[r] * a.sl2 : 0.f;
+  for (int r = 0; r < 4; ++r) {
+    const float inv = 1.f / l[r];
+#pragma unroll
+    for (int n = 0; n < C::NC; ++n) O[r][n] *= inv;
   }
   __syncthreads();
-  rows_softmax(pr, ld, a.T, nr, lse2);
-  rows_combine<D>(pr, ld, nr, a.Vc + hb, a.T, oc, part);
+  stage_rows<D>(Ks, O);
+  __syncthreads();
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
-    add_rows<D>(a.out, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.gamma);
+    add_rows<D>(a.out, (size_t)bh * a.L + sp.x, sp.y, Ks + r * C::LD, a.gamma);
   }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs a) {
+  using C = Tile<D>;
   extern __shared__ __align__(16) float sm[];
-  float* dO = sm;                          // [kRows][D] gamma * dout block sums (read as fragments)
-  float* oc = dO + kRows * D;              // [kRows][D] O_coarse rows, then dQc rows
-  float* part = oc + kRows * D;            // combine scratch
-  float* lse2 = part + kPartFloats<D>;     // [kRows]
-  float* pr = lse2 + kRows;                // [rows][ld] P, then dS; zero past T
-  const int bh = blockIdx.x, i0 = blockIdx.y * a.rows;
-  const int nr = min(a.rows, a.T - i0);
-  const int ld = (a.T + 3) & ~3;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* Qs = sm;
+  float* dOs = Qs + C::OP;   // dout block sums, then gamma * them
+  float* Ks = dOs + C::OP;
+  float* Vs = Ks + C::OP;
+  float* Ws = Vs + C::OP;    // dS tile
+  __shared__ float2 st[kBM];   // (lse2, Delta) of the CTA's rows
+  const int bh = blockIdx.y, i0 = blockIdx.x * kBM;
+  const int nr = min(kBM, a.T - i0);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
   const size_t hb = (size_t)bh * a.T * D;
-  // scores and softmax, as in the forward (Qc rows staged in dO's space)
-  for (int e = threadIdx.x; e < nr * D; e += kThreads) dO[e] = a.Qc[hb + (size_t)i0 * D + e];
-  __syncthreads();
-  for (int j = threadIdx.x; j < ld; j += kThreads) {
-    float acc[kRows];
-    if (j < a.T) row_dots<D>(dO, nr, a.Kc + hb + (size_t)j * D, acc);
-#pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < nr) pr[(size_t)r * ld + j] = j < a.T ? acc[r] * a.sl2 : 0.f;
-  }
-  __syncthreads();
-  rows_softmax(pr, ld, a.T, nr, lse2);
-  rows_combine<D>(pr, ld, nr, a.Vc + hb, a.T, oc, part);
-  // block sums of dout: thread = column, rows of block i0+r split over the thread slices
-  {
-    constexpr int SPLIT = kThreads / D;
-    const int d = threadIdx.x % D, h = threadIdx.x / D;
-    for (int r = 0; r < nr; ++r) {
+  load_tile<D>(Qs, a.Qc + hb, i0, a.T);
+  // block sums of dout: one (row, 8-column group) at a time, zero past T
+  for (int e = threadIdx.x; e < kBM * (D / 8); e += kThreads) {
+    const int r = e / (D / 8), c = (e % (D / 8)) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (r < nr) {
       const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
-      float acc = 0.f;
-      for (int t = h; t < sp.y; t += SPLIT) acc += __bfloat162float(a.dout[((size_t)bh * a.L + sp.x + t) * D + d]);
-      part[(h * kRows + r) * D + d] = acc;
+      const __nv_bfloat16* src = a.dout + ((size_t)bh * a.L + sp.x) * D + c;
+      for (int t = 0; t < sp.y; ++t) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + (size_t)t * D);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          acc[2 * k] += f.x;
+          acc[2 * k + 1] += f.y;
+        }
+      }
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < nr * D; e += kThreads) {
-      const int r = e / D, c = e % D;
-      float sum = 0.f;
-      for (int k = 0; k < SPLIT; ++k) sum += part[(k * kRows + r) * D + c];
-      dO[e] = sum;
-    }
-    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dOs[r * C::LD + c + k] = acc[k];
   }
-  // per row: g = (dout sum) . O (dgamma), then dO *= gamma, Delta = gamma g;
-  // one warp per row
-  if (warp < nr) {
+  // the forward again: lse2 and O of the CTA's rows
+  float m[4], l[4], O[4][C::NC];
+  flash_rows<D>(a, hb, Qs, Ks, Vs, m, l, O);
+  __syncthreads();   // dOs complete
+  float lse2[4], delta[4];
+  float gsum = 0.f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float inv = 1.f / l[r];
+    lse2[r] = m[r] + __log2f(l[r]);
     float g = 0.f;
-    for (int c = lane; c < D; c += 32) g = fmaf(dO[warp * D + c], oc[warp * D + c], g);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) g += __shfl_xor_sync(0xFFFFFFFFu, g, off);
-    for (int c = lane; c < D; c += 32) {
-      const float x = a.gamma * dO[warp * D + c];
-      dO[warp * D + c] = x;
-      a.dO[hb + (size_t)(i0 + warp) * D + c] = x;
-    }
-    if (lane == 0) {
-      a.stat[(size_t)bh * a.T + i0 + warp] = make_float2(lse2[warp], a.gamma * g);
-      if (a.dgamma) atomicAdd(a.dgamma + bh, g);
-      lse2[warp] = a.gamma * g;   // Delta of the row, for the dS pass
-    }
+    for (int gg = 0; gg < D / 64; ++gg)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) g = fmaf(dOs[(4 * ty + r) * C::LD + 4 * tx + 64 * gg + i], O[r][4 * gg + i] * inv, g);
+    g = row_sum16(g);   // (sum of the block's dout rows) . O_coarse
+    delta[r] = a.gamma * g;
+    if (4 * ty + r < nr) gsum += g;
+    if (tx == 0) st[4 * ty + r] = make_float2(lse2[r], delta[r]);
+  }
+  if (a.dgamma && tx == 0 && gsum != 0.f) atomicAdd(a.dgamma + bh, gsum);
+  __syncthreads();
+  // dO = gamma * sums, kept for the key pass with (lse2, Delta)
+  for (int e = threadIdx.x; e < kBM * D; e += kThreads) {
+    const int r = e / D, c = e % D;
+    const float x = a.gamma * dOs[r * C::LD + c];
+    dOs[r * C::LD + c] = x;
+    if (r < nr) a.dO[hb + (size_t)(i0 + r) * D + c] = x;
+  }
+  for (int r = threadIdx.x; r < nr; r += kThreads) a.stat[(size_t)bh * a.T + i0 + r] = st[r];
+  // dQc = s sum_j dS_j Kc_j
+  float dQ[4][C::NC];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int n = 0; n < C::NC; ++n) dQ[r][n] = 0.f;
+  for (int j0 = 0; j0 < a.T; j0 += kBM) {
+    __syncthreads();
+    load_tile<D>(Ks, a.Kc + hb, j0, a.T);
+    load_tile<D>(Vs, a.Vc + hb, j0, a.T);
+    __syncthreads();
+    float s[4][4], dp[4][4];
+    tile_dots<D>(Qs, Ks, s);
+    tile_dots<D>(dOs, Vs, dp);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float p = (j0 + tx + 16 * c < a.T) ? exp2f(s[r][c] * a.sl2 - lse2[r]) : 0.f;
+        s[r][c] = p * (dp[r][c] - delta[r]);
+      }
+    store_weights<D>(Ws, s);
+    __syncthreads();
+    tile_mul<D>(Ws, Ks, dQ);
   }
   __syncthreads();
-  // dS_rj = P_rj (dO_r . Vc_j - Delta_r), in place; one key block per thread
-  for (int j = threadIdx.x; j < a.T; j += kThreads) {
-    float dp[kRows];
-    row_dots<D>(dO, nr, a.Vc + hb + (size_t)j * D, dp);
-#pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < nr) pr[(size_t)r * ld + j] *= dp[r] - lse2[r];
-  }
+  stage_rows<D>(Ks, dQ);
   __syncthreads();
-  // dQc_r = s sum_j dS_rj Kc_j  -> dq rows of block i0+r += dQc_r / n
-  rows_combine<D>(pr, ld, nr, a.Kc + hb, a.T, oc, part);
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
-    add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, oc + r * D, a.scale / (float)sp.y);
+    add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, Ks + r * C::LD, a.scale / (float)sp.y);
   }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArgs a) {
+  using C = Tile<D>;
   extern __shared__ __align__(16) float sm[];
-  float* kc = sm;                          // [kRows][D] Kc rows, then dKc rows
-  float* vc = kc + kRows * D;              // [kRows][D] Vc rows, then dVc rows
-  float* part = vc + kRows * D;            // combine scratch
-  const int ld = (a.T + 3) & ~3;
-  float* pj = part + kPartFloats<D>;       // [rows][ld] P over query blocks, zero past T
-  float* sj = pj + (size_t)a.rows * ld;    // [rows][ld] dS, zero past T
-  const int bh = blockIdx.x, j0 = blockIdx.y * a.rows;
-  const int nr = min(a.rows, a.T - j0);
+  float* Ks = sm;            // this CTA's 64 key blocks (stationary); finally dKc rows
+  float* Vs = Ks + C::OP;    // their values; finally dVc rows
+  float* Qs = Vs + C::OP;    // a tile of 64 query blocks
+  float* dOs = Qs + C::OP;   // their gamma * dout sums
+  float* Ps = dOs + C::OP;   // P^T tile [key][query]
+  float* Ss = Ps + C::WP;    // dS^T tile
+  __shared__ float2 st[kBM];
+  const int bh = blockIdx.y, j0 = blockIdx.x * kBM;
+  const int nr = min(kBM, a.T - j0);
+  const int tx = threadIdx.x & 15;
   const size_t hb = (size_t)bh * a.T * D;
-  for (int e = threadIdx.x; e < nr * D; e += kThreads) {
-    kc[e] = a.Kc[hb + (size_t)j0 * D + e];
-    vc[e] = a.Vc[hb + (size_t)j0 * D + e];
-  }
-  __syncthreads();
-  // one query block per thread: its Qc and dO rows against all nr key blocks
-  for (int i = threadIdx.x; i < ld; i += kThreads) {
-    float s[kRows], dp[kRows];
-    float2 st = make_float2(0.f, 0.f);
-    if (i < a.T) {
-      row_dots<D>(kc, nr, a.Qc + hb + (size_t)i * D, s);
-      row_dots<D>(vc, nr, a.dO + hb + (size_t)i * D, dp);
-      st = a.stat[(size_t)bh * a.T + i];
-    }
+  load_tile<D>(Ks, a.Kc + hb, j0, a.T);
+  load_tile<D>(Vs, a.Vc + hb, j0, a.T);
+  float dK[4][C::NC], dV[4][C::NC];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      if (r < nr) {
-        const float p = i < a.T ? exp2f(s[r] * a.sl2 - st.x) : 0.f;
-        pj[(size_t)r * ld + i] = p;
-        sj[(size_t)r * ld + i] = i < a.T ? p * (dp[r] - st.y) : 0.f;
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int n = 0; n < C::NC; ++n) dK[r][n] = dV[r][n] = 0.f;
+  for (int i0 = 0; i0 < a.T; i0 += kBM) {
+    __syncthreads();
+    load_tile<D>(Qs, a.Qc + hb, i0, a.T);
+    load_tile<D>(dOs, a.dO + hb, i0, a.T);
+    for (int r = threadIdx.x; r < kBM; r += kThreads)
+      st[r] = i0 + r < a.T ? a.stat[(size_t)bh * a.T + i0 + r] : make_float2(INFINITY, 0.f);
+    __syncthreads();
+    float s[4][4], dp[4][4];
+    tile_dots<D>(Ks, Qs, s);    // S^T: key rows, query columns tx + 16 c
+    tile_dots<D>(Vs, dOs, dp);  // dP^T
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float2 q = st[tx + 16 * c];   // lse2 = inf past T: P = 0
+        const float p = exp2f(s[r][c] * a.sl2 - q.x);
+        s[r][c] = p;
+        dp[r][c] = p * (dp[r][c] - q.y);
       }
-    }
+    store_weights<D>(Ps, s);
+    store_weights<D>(Ss, dp);
+    __syncthreads();
+    tile_mul<D>(Ps, dOs, dV);
+    tile_mul<D>(Ss, Qs, dK);
   }
   __syncthreads();
-  // dKc_r = s sum_i dS_ri Qc_i, dVc_r = sum_i P_ri dO_i
-  rows_combine<D>(sj, ld, nr, a.Qc + hb, a.T, kc, part);
-  rows_combine<D>(pj, ld, nr, a.dO + hb, a.T, vc, part);
+  stage_rows<D>(Ks, dK);
+  stage_rows<D>(Vs, dV);
+  __syncthreads();
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(j0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
-    add_rows<D>(a.dk, (size_t)bh * a.L + sp.x, sp.y, kc + r * D, a.scale / (float)sp.y);
-    add_rows<D>(a.dv, (size_t)bh * a.L + sp.x, sp.y, vc + r * D, 1.f / (float)sp.y);
+    add_rows<D>(a.dk, (size_t)bh * a.L + sp.x, sp.y, Ks + r * C::LD, a.scale / (float)sp.y);
+    add_rows<D>(a.dv, (size_t)bh * a.L + sp.x, sp.y, Vs + r * C::LD, 1.f / (float)sp.y);
   }
 }
 
-// Shared-memory bytes of each kernel for `rows` blocks per CTA.
 template <int D>
-size_t fwd_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + kRows + (size_t)rows * ((T + 3) & ~3)) * 4; }
+constexpr size_t fwd_smem() { return (size_t)3 * Tile<D>::OP * 4; }
 template <int D>
-size_t kv_smem(int T, int rows) { return (size_t)(kVecFloats<D> + kPartFloats<D> + 2 * (size_t)rows * ((T + 3) & ~3)) * 4; }
-
-constexpr size_t kSmemBudget = 160 * 1024;
+constexpr size_t bwd_q_smem() { return ((size_t)4 * Tile<D>::OP + Tile<D>::WP) * 4; }
+template <int D>
+constexpr size_t bwd_kv_smem() { return ((size_t)4 * Tile<D>::OP + 2 * Tile<D>::WP) * 4; }
 
 template <int D>
 static cudaError_t launch_t(const Dims& d, CoarseArgs a, bool backward, cudaStream_t st) {
   static std::atomic<unsigned long long> attr_done{0};   // per template instance
   {
     const cudaError_t e = once_per_device(attr_done, [] {
-      cudaError_t r = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+      cudaError_t r = cudaFuncSetAttribute(coarse_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D>());
       if (r == cudaSuccess)
-        r = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+        r = cudaFuncSetAttribute(coarse_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_q_smem<D>());
       if (r == cudaSuccess)
-        r = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+        r = cudaFuncSetAttribute(coarse_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_kv_smem<D>());
       return r;
     });
     if (e != cudaSuccess) return e;
   }
-  // as many blocks per CTA as the score rows leave room for (at most kRows)
-  int rq = kRows;
-  while (rq > 1 && fwd_smem<D>(d.T, rq) > kSmemBudget) --rq;
-  a.rows = rq;
-  const dim3 gq(d.BH, (d.T + rq - 1) / rq);
+  const dim3 grid((d.T + kBM - 1) / kBM, d.BH);
   if (!backward) {
-    coarse_fwd_kernel<D><<<gq, kThreads, fwd_smem<D>(d.T, rq), st>>>(a);
+    coarse_fwd_kernel<D><<<grid, kThreads, fwd_smem<D>(), st>>>(a);
     return cudaGetLastError();
   }
-  coarse_bwd_q_kernel<D><<<gq, kThreads, fwd_smem<D>(d.T, rq), st>>>(a);
+  coarse_bwd_q_kernel<D><<<grid, kThreads, bwd_q_smem<D>(), st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int rk = kRows;
-  while (rk > 1 && kv_smem<D>(d.T, rk) > kSmemBudget) --rk;
-  a.rows = rk;
-  coarse_bwd_kv_kernel<D><<<dim3(d.BH, (d.T + rk - 1) / rk), kThreads, kv_smem<D>(d.T, rk), st>>>(a);
+  coarse_bwd_kv_kernel<D><<<grid, kThreads, bwd_kv_smem<D>(), st>>>(a);
   return cudaGetLastError();
 }
 
