@@ -18,7 +18,9 @@
 // 4 x 4 micro-tile of each 64 x 64 score tile (rows 4 ty .. 4 ty + 3, columns
 // tx, tx + 16, tx + 32, tx + 48) and 4 rows x D/16 columns of each 64 x D
 // product; softmax rows run online (running maximum and sum), as in flash
-// attention:
+// attention.  The backward kernels copy the next tile pair in with cp.async
+// while they use the current one (one CTA per SM either way); the forward
+// keeps one pair, so that two CTAs fit on an SM:
 //   coarse_fwd_kernel    O_coarse of 64 query blocks -> out rows += gamma O_i
 //   coarse_bwd_q_kernel  per query block i: the forward again (lse2_i, O_i),
 //                        dO_i = gamma * sum of the block's dout rows, Delta_i =
@@ -70,6 +72,28 @@ __device__ void load_tile(float* Xs, const float* __restrict__ X, int r0, int n)
     if (r0 + r < n) v = *reinterpret_cast<const float4*>(X + (size_t)(r0 + r) * D + 4 * c4);
     *reinterpret_cast<float4*>(Xs + r * Tile<D>::LD + 4 * c4) = v;
   }
+}
+
+// The same as an asynchronous copy (cp.async, 16 bytes a piece; rows past n
+// are filled with zeros by a source size of 0).  The caller commits the
+// group and waits for it.
+template <int D>
+__device__ __forceinline__ void load_tile_async(float* Xs, const float* __restrict__ X, int r0, int n) {
+  constexpr int V4 = D / 4;
+  for (int e = threadIdx.x; e < kBM * V4; e += kThreads) {
+    const int r = e / V4, c4 = e % V4;
+    const bool ok = r0 + r < n;
+    const float* src = X + (size_t)(ok ? r0 + r : 0) * D + 4 * c4;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(Xs + r * Tile<D>::LD + 4 * c4)),
+                 "l"(src), "r"(ok ? 16 : 0)
+                 : "memory");
+  }
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most N of this thread's committed groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // acc[a][c] = A[4 ty + a] . B[tx + 16 c] over D (A, B: 64 x LD tiles)
@@ -151,11 +175,14 @@ __device__ __forceinline__ float row_sum16(float x) {
   return x;
 }
 
-// The forward of this CTA's 64 query rows (Qs) over all T keys: running
-// maximum m and sum l (log2 units) per row and the unnormalised O.  Uses Ks
-// (then the weight tile) and Vs as scratch.
+// The forward of this CTA's 64 query rows (Qs) over all T keys, one (K, V)
+// tile pair at a time: running maximum m and sum l (log2 units) per row and
+// the unnormalised O.  Uses Ks (then the weight tile) and Vs as scratch.
+// The forward kernel takes this form: with one tile pair it holds 99 KB of
+// shared memory at D=128 and two CTAs fit on an SM, which beat one CTA with
+// the next pair prefetched.
 template <int D>
-__device__ void flash_rows(const CoarseArgs& a, size_t hb, const float* Qs, float* Ks, float* Vs, float (&m)[4],
+__device__ void flash_rows_sync(const CoarseArgs& a, size_t hb, const float* Qs, float* Ks, float* Vs, float (&m)[4],
                            float (&l)[4], float (&O)[4][Tile<D>::NC]) {
   const int tx = threadIdx.x & 15;
 #pragma unroll
@@ -200,6 +227,68 @@ __device__ void flash_rows(const CoarseArgs& a, size_t hb, const float* Qs, floa
   }
 }
 
+// The forward of this CTA's 64 query rows (Qs) over all T keys: running
+// maximum m and sum l (log2 units) per row and the unnormalised O.  KV holds
+// two (K, V) tile pairs: the next pair is copied in while the current one is
+// used, and the current K tile takes the weights once its scores are formed.
+template <int D>
+__device__ void flash_rows(const CoarseArgs& a, size_t hb, const float* Qs, float* KV, float (&m)[4], float (&l)[4],
+                           float (&O)[4][Tile<D>::NC]) {
+  using C = Tile<D>;
+  const int tx = threadIdx.x & 15;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.f;
+#pragma unroll
+    for (int n = 0; n < C::NC; ++n) O[r][n] = 0.f;
+  }
+  __syncthreads();   // the buffers' previous users are done
+  load_tile_async<D>(KV, a.Kc + hb, 0, a.T);
+  load_tile_async<D>(KV + C::OP, a.Vc + hb, 0, a.T);
+  cp_async_commit();
+  for (int j0 = 0, u = 0; j0 < a.T; j0 += kBM, u ^= 1) {
+    float* Ks = KV + 2 * u * C::OP;
+    float* Vs = Ks + C::OP;
+    if (j0 + kBM < a.T) {   // the next pair into the other buffers (free since the end of the last tile)
+      load_tile_async<D>(KV + 2 * (u ^ 1) * C::OP, a.Kc + hb, j0 + kBM, a.T);
+      load_tile_async<D>(KV + (2 * (u ^ 1) + 1) * C::OP, a.Vc + hb, j0 + kBM, a.T);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();   // this tile's pair has landed (this thread's part)
+    __syncthreads();      // and every thread's
+    float s[4][4];
+    tile_dots<D>(Qs, Ks, s);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float cm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[r][c] = (j0 + tx + 16 * c < a.T) ? s[r][c] * a.sl2 : -INFINITY;
+        cm = fmaxf(cm, s[r][c]);
+      }
+      const float mn = fmaxf(m[r], row_max16(cm));   // finite: key j0 + 0 < T
+      const float alpha = exp2f(m[r] - mn);           // 0 on the first tile
+      float ps = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[r][c] = exp2f(s[r][c] - mn);
+        ps += s[r][c];
+      }
+      l[r] = l[r] * alpha + row_sum16(ps);
+      m[r] = mn;
+#pragma unroll
+      for (int n = 0; n < C::NC; ++n) O[r][n] *= alpha;
+    }
+    __syncthreads();   // every thread has read Ks: the weights take its place
+    store_weights<D>(Ks, s);
+    __syncthreads();
+    tile_mul<D>(Ks, Vs, O);
+    __syncthreads();   // the pair's buffers may take the pair after next
+  }
+  cp_async_wait<0>();
+}
+
 // Xs (64 x LD) = the thread's 4 x NC values (rows 4 ty + r, columns 4 tx + 64 g + i)
 template <int D>
 __device__ __forceinline__ void stage_rows(float* Xs, const float (&v)[4][Tile<D>::NC]) {
@@ -241,7 +330,7 @@ __global__ void __launch_bounds__(kThreads) coarse_fwd_kernel(const CoarseArgs a
   const size_t hb = (size_t)bh * a.T * D;
   load_tile<D>(Qs, a.Qc + hb, i0, a.T);
   float m[4], l[4], O[4][C::NC];
-  flash_rows<D>(a, hb, Qs, Ks, Vs, m, l, O);
+  flash_rows_sync<D>(a, hb, Qs, Ks, Vs, m, l, O);
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const float inv = 1.f / l[r];
@@ -258,14 +347,13 @@ __global__ void __launch_bounds__(kThreads) coarse_fwd_kernel(const CoarseArgs a
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) coarse_bwd_q_kernel(const CoarseArgs a) {
   using C = Tile<D>;
   extern __shared__ __align__(16) float sm[];
   float* Qs = sm;
   float* dOs = Qs + C::OP;   // dout block sums, then gamma * them
-  float* Ks = dOs + C::OP;
-  float* Vs = Ks + C::OP;
-  float* Ws = Vs + C::OP;    // dS tile
+  float* KV = dOs + C::OP;   // two (K, V) tile pairs
+  float* Ws = KV + 4 * C::OP;   // dS tile
   __shared__ float2 st[kBM];   // (lse2, Delta) of the CTA's rows
   const int bh = blockIdx.y, i0 = blockIdx.x * kBM;
   const int nr = min(kBM, a.T - i0);
@@ -295,7 +383,7 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs
   }
   // the forward again: lse2 and O of the CTA's rows
   float m[4], l[4], O[4][C::NC];
-  flash_rows<D>(a, hb, Qs, Ks, Vs, m, l, O);
+  flash_rows<D>(a, hb, Qs, KV, m, l, O);
   __syncthreads();   // dOs complete
   float lse2[4], delta[4];
   float gsum = 0.f;
@@ -329,10 +417,19 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int n = 0; n < C::NC; ++n) dQ[r][n] = 0.f;
-  for (int j0 = 0; j0 < a.T; j0 += kBM) {
-    __syncthreads();
-    load_tile<D>(Ks, a.Kc + hb, j0, a.T);
-    load_tile<D>(Vs, a.Vc + hb, j0, a.T);
+  __syncthreads();   // dOs scaled; the flash pass's buffers are free
+  load_tile_async<D>(KV, a.Kc + hb, 0, a.T);
+  load_tile_async<D>(KV + C::OP, a.Vc + hb, 0, a.T);
+  cp_async_commit();
+  for (int j0 = 0, u = 0; j0 < a.T; j0 += kBM, u ^= 1) {
+    float* Ks = KV + 2 * u * C::OP;
+    float* Vs = Ks + C::OP;
+    if (j0 + kBM < a.T) {
+      load_tile_async<D>(KV + 2 * (u ^ 1) * C::OP, a.Kc + hb, j0 + kBM, a.T);
+      load_tile_async<D>(KV + (2 * (u ^ 1) + 1) * C::OP, a.Vc + hb, j0 + kBM, a.T);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
     float s[4][4], dp[4][4];
     tile_dots<D>(Qs, Ks, s);
@@ -347,13 +444,14 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_q_kernel(const CoarseArgs
     store_weights<D>(Ws, s);
     __syncthreads();
     tile_mul<D>(Ws, Ks, dQ);
+    __syncthreads();   // Ws and this pair's buffers are free again
   }
-  __syncthreads();
-  stage_rows<D>(Ks, dQ);
+  cp_async_wait<0>();
+  stage_rows<D>(KV, dQ);
   __syncthreads();
   for (int r = 0; r < nr; ++r) {
     const int2 sp = block_span(i0 + r, a.L_src, a.L_ctx, a.b, a.T_src);
-    add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, Ks + r * C::LD, a.scale / (float)sp.y);
+    add_rows<D>(a.dq, (size_t)bh * a.L + sp.x, sp.y, KV + r * C::LD, a.scale / (float)sp.y);
   }
 }
 
@@ -363,11 +461,9 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
   extern __shared__ __align__(16) float sm[];
   float* Ks = sm;            // this CTA's 64 key blocks (stationary); finally dKc rows
   float* Vs = Ks + C::OP;    // their values; finally dVc rows
-  float* Qs = Vs + C::OP;    // a tile of 64 query blocks
-  float* dOs = Qs + C::OP;   // their gamma * dout sums
-  float* Ps = dOs + C::OP;   // P^T tile [key][query]
-  float* Ss = Ps + C::WP;    // dS^T tile
-  __shared__ float2 st[kBM];
+  float* QD = Vs + C::OP;    // two (Qc, gamma * dout sums) tile pairs of 64 query blocks
+  float* Ws = QD + 4 * C::OP;   // P^T, then dS^T [key][query]
+  __shared__ float2 st[2][kBM];
   const int bh = blockIdx.y, j0 = blockIdx.x * kBM;
   const int nr = min(kBM, a.T - j0);
   const int tx = threadIdx.x & 15;
@@ -379,12 +475,24 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int n = 0; n < C::NC; ++n) dK[r][n] = dV[r][n] = 0.f;
-  for (int i0 = 0; i0 < a.T; i0 += kBM) {
-    __syncthreads();
-    load_tile<D>(Qs, a.Qc + hb, i0, a.T);
-    load_tile<D>(dOs, a.dO + hb, i0, a.T);
-    for (int r = threadIdx.x; r < kBM; r += kThreads)
-      st[r] = i0 + r < a.T ? a.stat[(size_t)bh * a.T + i0 + r] : make_float2(INFINITY, 0.f);
+  auto load_pair = [&](int i0, int u) {
+    load_tile_async<D>(QD + 2 * u * C::OP, a.Qc + hb, i0, a.T);
+    load_tile_async<D>(QD + (2 * u + 1) * C::OP, a.dO + hb, i0, a.T);
+    for (int r = threadIdx.x; r < kBM; r += kThreads) {
+      const bool ok = i0 + r < a.T;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(&st[u][r])),
+                   "l"(a.stat + (size_t)bh * a.T + (ok ? i0 + r : 0)), "r"(ok ? 8 : 0)
+                   : "memory");
+    }
+  };
+  load_pair(0, 0);
+  cp_async_commit();
+  for (int i0 = 0, u = 0; i0 < a.T; i0 += kBM, u ^= 1) {
+    const float* Qs = QD + 2 * u * C::OP;
+    const float* dOs = Qs + C::OP;
+    if (i0 + kBM < a.T) load_pair(i0 + kBM, u ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
     float s[4][4], dp[4][4];
     tile_dots<D>(Ks, Qs, s);    // S^T: key rows, query columns tx + 16 c
@@ -393,17 +501,22 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
     for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float2 q = st[tx + 16 * c];   // lse2 = inf past T: P = 0
-        const float p = exp2f(s[r][c] * a.sl2 - q.x);
+        const int qi = tx + 16 * c;
+        const float2 q = st[u][qi];
+        const float p = i0 + qi < a.T ? exp2f(s[r][c] * a.sl2 - q.x) : 0.f;
         s[r][c] = p;
         dp[r][c] = p * (dp[r][c] - q.y);
       }
-    store_weights<D>(Ps, s);
-    store_weights<D>(Ss, dp);
+    store_weights<D>(Ws, s);
     __syncthreads();
-    tile_mul<D>(Ps, dOs, dV);
-    tile_mul<D>(Ss, Qs, dK);
+    tile_mul<D>(Ws, dOs, dV);
+    __syncthreads();   // P^T read: dS^T takes its place
+    store_weights<D>(Ws, dp);
+    __syncthreads();
+    tile_mul<D>(Ws, Qs, dK);
+    __syncthreads();   // this pair's buffers and Ws are free again
   }
+  cp_async_wait<0>();
   __syncthreads();
   stage_rows<D>(Ks, dK);
   stage_rows<D>(Vs, dV);
@@ -418,9 +531,9 @@ __global__ void __launch_bounds__(kThreads) coarse_bwd_kv_kernel(const CoarseArg
 template <int D>
 constexpr size_t fwd_smem() { return (size_t)3 * Tile<D>::OP * 4; }
 template <int D>
-constexpr size_t bwd_q_smem() { return ((size_t)4 * Tile<D>::OP + Tile<D>::WP) * 4; }
+constexpr size_t bwd_q_smem() { return ((size_t)6 * Tile<D>::OP + Tile<D>::WP) * 4; }
 template <int D>
-constexpr size_t bwd_kv_smem() { return ((size_t)4 * Tile<D>::OP + 2 * Tile<D>::WP) * 4; }
+constexpr size_t bwd_kv_smem() { return ((size_t)6 * Tile<D>::OP + Tile<D>::WP) * 4; }
 
 template <int D>
 static cudaError_t launch_t(const Dims& d, CoarseArgs a, bool backward, cudaStream_t st) {
