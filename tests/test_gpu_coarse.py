@@ -35,8 +35,11 @@ def assert_close(got, ref, what):
     assert np.all(e <= bound), (what, float((e - bound).max()), int((e > bound).sum()))
 
 
+# the last one has 1100 pooled blocks in its head: 17 full 64-block tiles
+# and a ragged one, on both sides of the kernels' tile loops
 CASES = [("d128_b64", 1, 2, 128, 520, 300, 64, 0.7), ("d128_b32", 1, 2, 128, 333, 200, 32, -1.5),
-         ("d64_b64", 2, 1, 64, 700, 333, 64, 0.25), ("d64_b32_one_ctx_token", 1, 2, 64, 257, 1, 32, 2.0)]
+         ("d64_b64", 2, 1, 64, 700, 333, 64, 0.25), ("d64_b32_one_ctx_token", 1, 2, 64, 257, 1, 32, 2.0),
+         ("d128_b32_1100_blocks", 1, 1, 128, 17600, 17600, 32, 0.5)]
 
 
 @pytest.mark.parametrize("name,B,H,D,Ls,Lc,b,gamma", CASES)
