@@ -370,9 +370,9 @@ static isa_status run_attention(const Dims& d, int mode, const void* q, const vo
   return ISA_OK;
 }
 
-// Byte offsets of the backward workspace: (lse2, Delta) per row of every
-// query block ([BH, T, b], padded past each block's end), then
-// the fp32 gradients of the pooled keys and values.
+// Byte offsets of the backward workspace: lse2 and Delta per row of every
+// query block ([BH, T, 2, b] fp32, padded past each block's end), then the
+// fp32 gradients of the pooled keys and values.
 struct BwdLayout {
   size_t dl, dKc, dVc, total;
 };
@@ -466,7 +466,7 @@ isa_status isa_backward(const isa_params* p, const void* q, const void* k, const
   b.dout = static_cast<const __nv_bfloat16*>(dout);
   b.lse = lse;
   char* w = static_cast<char*>(bws);
-  b.dl = reinterpret_cast<float2*>(w + BL.dl);
+  b.dl = reinterpret_cast<float*>(w + BL.dl);
   b.dKc = reinterpret_cast<float*>(w + BL.dKc);
   b.dVc = reinterpret_cast<float*>(w + BL.dVc);
   b.dq = static_cast<__nv_bfloat16*>(dq);

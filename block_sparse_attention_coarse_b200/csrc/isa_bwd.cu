@@ -52,13 +52,14 @@ __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
   return acc;
 }
 
-// dl[(bh*T + j)*b + r] = (lse * log2 e, sum_d dout * o) of row r of block j
-// of head bh, and (inf, 0) for r past the block's end, so that every query
-// block's entries are one aligned run of b float2.  D/8 lanes per entry,
+// dl[((bh*T + j)*2 + 0)*b + r] = lse * log2 e and dl[((bh*T + j)*2 + 1)*b + r]
+// = sum_d dout * o of row r of block j of head bh, and (inf, 0) for r past
+// the block's end: every query block's entries are a run of b lse2 values
+// followed by a run of b Delta values.  D/8 lanes per entry,
 // grid-stride over the BH*T*b entries (the loop bound is warp-uniform).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
-                                                       const float* __restrict__ lse, float2* __restrict__ dl,
+                                                       const float* __restrict__ lse, float* __restrict__ dl,
                                                        int T, int b, int L, int L_src, int L_ctx, int T_src,
                                                        size_t entries) {
   constexpr int LPR = D / 8;
@@ -81,7 +82,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__
     if (valid) acc = dot_bf16x8(o[row * LPR + lane % LPR], dout[row * LPR + lane % LPR]);
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-    if (e < entries && lane % LPR == 0) dl[e] = valid ? make_float2(lse[row] * kLog2e, acc) : make_float2(INFINITY, 0.f);
+    if (e < entries && lane % LPR == 0) {
+      const size_t blk = e / b, r = e % b;   // (bh*T + j), row in the block
+      dl[(blk * 2) * b + r] = valid ? lse[row] * kLog2e : INFINITY;
+      dl[(blk * 2 + 1) * b + r] = valid ? acc : 0.f;
+    }
   }
 }
 
@@ -165,7 +170,7 @@ struct KvCfg {
   static constexpr uint32_t V_OFF = TILE;
   static constexpr uint32_t Q_OFF = 2 * TILE;
   static constexpr uint32_t DO_OFF = Q_OFF + kNSQ * TILE;
-  static constexpr uint32_t DL_OFF = DO_OFF + kNSQ * TILE;   // (lse2, Delta) of the 128 step rows
+  static constexpr uint32_t DL_OFF = DO_OFF + kNSQ * TILE;   // lse2 and Delta runs of the step's query blocks
   static constexpr uint32_t DL_STAGE = 128 * 8;
   static constexpr uint32_t SMEM_USED = DL_OFF + kNSQ * DL_STAGE + 1024;
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits on an SM
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         for (int g = 0; g < GQ; ++g) {
           const int row = bh * a.L + (m.cnt[g] > 0 ? m.start[g] : 0);
           bulk_load_1d(sgen + C::DL_OFF + s * C::DL_STAGE + g * R * 8,
-                       b.dl + ((size_t)bh * (a.T_src + a.T_ctx) + m.blk[g]) * R, R * 8, &q_full[s]);
+                       b.dl + ((size_t)bh * (a.T_src + a.T_ctx) + m.blk[g]) * 2 * R, R * 8, &q_full[s]);
           for (int c = 0; c < C::NCH; ++c) {
             tma_load_2d(sgen + C::Q_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, &tm_q, c * 64, row, &q_full[s]);
             tma_load_2d(sgen + C::DO_OFF + s * C::TILE + c * C::CHUNK + g * C::BOX, &tm_do, c * 64, row,
@@ -522,32 +527,36 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc_fence_after();
         const int last = meta[s].last;
         const bool on = row_valid && ((meta[s].m[gq][r >> 5] >> (r & 31)) & 1u);
-        // (lse2, Delta) of this warp's 32 columns, two columns per 16-byte
-        // broadcast load; rows past a block's end hold (inf, 0), so P = 0 there
-        const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE) + c0 / 2;
-        // phase A: P^T, 16 columns at a time
+        // lse2 and Delta of this warp's 32 columns (one query block's rows
+        // c0 % R .. +31), four columns per 16-byte broadcast load; rows past a
+        // block's end hold (inf, 0), so P = 0 there
+        const float4* dls = reinterpret_cast<const float4*>(sgen + C::DL_OFF + s * C::DL_STAGE +
+                                                            (gq * 2 * R + c0 % R) * 4);
+        // phase A: P^T of the 32 columns, loaded in one TMEM round trip
         float p[32];
+        {
+          uint32_t sv[2][16];
+          tmem_ld16_pair_sync(tl + kTST + c0, sv[0], tl + kTST + c0 + 16, sv[1]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float2 lz[8];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 x = dls[8 * h + e];
-            lz[e] = make_float2(bias - x.x, bias - x.z);
+            for (int e = 0; e < 16; e += 4) {
+              const float4 l4 = dls[(16 * h + e) >> 2];
+              float p0 = ex2(fmaf(__uint_as_float(sv[h][e]), sl2, bias - l4.x));
+              float p1 = ex2(fmaf(__uint_as_float(sv[h][e + 1]), sl2, bias - l4.y));
+              float p2 = ex2(fmaf(__uint_as_float(sv[h][e + 2]), sl2, bias - l4.z));
+              float p3 = ex2(fmaf(__uint_as_float(sv[h][e + 3]), sl2, bias - l4.w));
+              if (!on) p0 = p1 = p2 = p3 = 0.f;
+              p[16 * h + e] = p0;
+              p[16 * h + e + 1] = p1;
+              p[16 * h + e + 2] = p2;
+              p[16 * h + e + 3] = p3;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+              pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+            }
+            tmem_st8(tl + kTST + c0 + 16 * h, pk);
           }
-          uint32_t sv[16];
-          tmem_ld16_sync(tl + kTST + c0 + 16 * h, sv);
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float p0 = ex2(fmaf(__uint_as_float(sv[e]), sl2, lz[e >> 1].x));
-            float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), sl2, lz[e >> 1].y));
-            if (!on) p0 = p1 = 0.f;
-            p[16 * h + e] = p0;
-            p[16 * h + e + 1] = p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st8(tl + kTST + c0 + 16 * h, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -559,24 +568,25 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           break;
         }
         tc_fence_after();
+        {
+          const float4* dds = dls + R / 4;   // Delta of the same columns
+          uint32_t dp[2][16];
+          tmem_ld16_pair_sync(tl + kTDP + c0, dp[0], tl + kTDP + c0 + 16, dp[1]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float2 dz[8];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pd[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 x = dls[8 * h + e];
-            dz[e] = make_float2(x.y, x.w);
+            for (int e = 0; e < 16; e += 4) {
+              const float4 d4 = dds[(16 * h + e) >> 2];
+              const float g0 = p[16 * h + e] * (__uint_as_float(dp[h][e]) - d4.x);
+              const float g1 = p[16 * h + e + 1] * (__uint_as_float(dp[h][e + 1]) - d4.y);
+              const float g2 = p[16 * h + e + 2] * (__uint_as_float(dp[h][e + 2]) - d4.z);
+              const float g3 = p[16 * h + e + 3] * (__uint_as_float(dp[h][e + 3]) - d4.w);
+              pd[e >> 1] = pack_bf16x2(g0, g1);
+              pd[(e >> 1) + 1] = pack_bf16x2(g2, g3);
+            }
+            tmem_st8(tl + kTDP + c0 + 16 * h, pd);
           }
-          uint32_t dp[16];
-          tmem_ld16_sync(tl + kTDP + c0 + 16 * h, dp);
-          uint32_t pd[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const float g0 = p[16 * h + e] * (__uint_as_float(dp[e]) - dz[e >> 1].x);
-            const float g1 = p[16 * h + e + 1] * (__uint_as_float(dp[e + 1]) - dz[e >> 1].y);
-            pd[e >> 1] = pack_bf16x2(g0, g1);
-          }
-          tmem_st8(tl + kTDP + c0 + 16 * h, pd);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -883,8 +893,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const bool row_valid = rr < qs.y;
       const size_t tok = (size_t)I.bh * a.L + qs.x + rr;
       const int qblk = qs.x < a.L_src ? qs.x / a.b : a.T_src + (qs.x - a.L_src) / a.b;
-      const float2 mine = row_valid ? b.dl[((size_t)I.bh * (a.T_src + a.T_ctx) + qblk) * a.b + rr]
-                                    : make_float2(INFINITY, 0.f);
+      const size_t dli = (((size_t)I.bh * (a.T_src + a.T_ctx) + qblk) * 2) * a.b + rr;
+      const float2 mine = row_valid ? make_float2(b.dl[dli], b.dl[dli + a.b]) : make_float2(INFINITY, 0.f);
       const uint32_t* rbits = nullptr;
       int pb0 = -1, pb1 = -1;
       float d0 = 0.f, d1 = 0.f;

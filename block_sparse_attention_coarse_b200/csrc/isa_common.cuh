@@ -63,7 +63,8 @@ struct BwdArgs {
   const __nv_bfloat16* o;      // forward output [BH*L, D]
   const __nv_bfloat16* dout;   // gradient of the output [BH*L, D]
   const float* lse;            // forward natural-log normalisers [BH*L]
-  float2* dl;                  // [BH, T, b] per block row: (lse * log2 e, rowsum(dout * o)); (inf, 0) past a block's end
+  float* dl;                   // [BH, T, 2, b]: per block, the rows' lse * log2 e, then their rowsum(dout * o);
+                               // (inf, 0) past a block's end
   float* dKc;                  // [BH, T_kv_pad, D] gradient of the pooled keys (scaled)
   float* dVc;                  // [BH, T_kv_pad, D] gradient of the pooled values
   __nv_bfloat16 *dq, *dk, *dv; // [BH*L, D]
