@@ -417,10 +417,68 @@ __device__ __forceinline__ uint32_t f2ord(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The k-th largest of key[0..n) as an order key (f2ord), 1 <= k <= n, by one
+// warp: a radix select over the order keys, 8 bits per pass from the top,
+// with a 256-bin histogram per pass in `hist` (shared memory, 256 words,
+// this warp's alone).  Each pass counts the keys that match the digits
+// chosen so far; the lanes scan the bins from the top digit down (lane l
+// holds bins 255-8l .. 248-8l) and keep the digit at which the running count
+// reaches the remaining rank.
+__device__ inline uint32_t warp_kth_largest(const float* key, int n, int k, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  uint32_t kk = (uint32_t)k;   // rank of the wanted key among those matching prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0u;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t o = f2ord(key[i]);
+      if ((o & pmask) == prefix) atomicAdd(&hist[(o >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    uint32_t c[8], sum = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[j] = hist[255 - 8 * lane - j];
+      sum += c[j];
+    }
+    uint32_t incl = sum;   // keys in the bins of lanes 0..lane (digits from the top)
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, excl < kk && kk <= incl)) - 1;
+    int d = 0;
+    uint32_t above = 0u;
+    if (lane == src) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (run + c[j] >= kk) {
+          d = 255 - 8 * lane - j;
+          above = run;
+          break;
+        }
+        run += c[j];
+      }
+    }
+    d = __shfl_sync(0xFFFFFFFFu, d, src);
+    above = __shfl_sync(0xFFFFFFFFu, above, src);
+    prefix |= (uint32_t)d << shift;
+    pmask |= 255u << shift;
+    kk -= above;
+    __syncwarp();   // every lane has read the bins before the next pass clears them
+  }
+  return prefix;
+}
+
 // One warp selects the k largest of key[0..n) (shared memory), ties to the
 // lower index, writing the chosen indices in ascending order to out[0..k)
 // and, when bits != nullptr, the selection as a bitmap of ceil(n/32) words.
-__device__ inline void warp_topk(const float* key, int n, int k, int* out, uint32_t* bits) {
+// hist: 256 words of shared memory for this warp alone.
+__device__ inline void warp_topk(const float* key, int n, int k, int* out, uint32_t* bits, uint32_t* hist) {
   const int lane = threadIdx.x & 31;
   if (k >= n) {
     for (int i = lane; i < n; i += 32) out[i] = i;
@@ -431,17 +489,8 @@ __device__ inline void warp_topk(const float* key, int n, int k, int* out, uint3
       }
     return;
   }
-  uint32_t t = 0;
-  if (k > 0) {
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = t | (1u << bit);
-      int c = 0;
-#pragma unroll 4
-      for (int i = lane; i < n; i += 32) c += f2ord(key[i]) >= cand;
-      c = __reduce_add_sync(0xFFFFFFFFu, c);
-      if (c >= k) t = cand;
-    }
-  }
+  // t: the k-th largest order key (0 when k == 0: nothing is selected)
+  const uint32_t t = k > 0 ? warp_kth_largest(key, n, k, hist) : 0u;
   int gt = 0;
   if (k > 0) {
 #pragma unroll 4

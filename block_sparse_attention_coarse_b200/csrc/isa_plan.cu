@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(256) ctx_select_kernel(Dims dm, PlanPtrs pp) {
   float* imp = sm + D;            // [T_ctx]
   int* sel = reinterpret_cast<int*>(imp + dm.T_ctx);   // [K_sel]
   __shared__ float part[256];
+  __shared__ uint32_t hist[256];   // the selection's radix histogram
   const int bh = blockIdx.x, tid = threadIdx.x;
   const float* Qc = pp.Qc + (size_t)bh * dm.T * D;
   const float* Kc = pp.Kc + (size_t)bh * dm.T * D;
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(256) ctx_select_kernel(Dims dm, PlanPtrs pp) {
     }
   }
   __syncthreads();
-  if (warp == 0) warp_topk(imp, dm.T_ctx, dm.K_sel, sel, nullptr);
+  if (warp == 0) warp_topk(imp, dm.T_ctx, dm.K_sel, sel, nullptr, hist);
   __syncthreads();
   int* kept = pp.kept + (size_t)bh * dm.T_kv;
   for (int i = tid; i < dm.K_sel; i += 256) pp.ctx_sel[(size_t)bh * dm.K_sel + i] = sel[i];
@@ -311,10 +312,11 @@ __global__ void __launch_bounds__(256) split_kernel(Dims dm, PlanPtrs pp) {
   float* E = sm;                                  // [T]
   int* sharp = reinterpret_cast<int*>(E + dm.T);  // [n_sharp]
   uint32_t* bits = reinterpret_cast<uint32_t*>(sharp + dm.n_sharp);   // [ceil(T/32)]
+  __shared__ uint32_t hist[256];   // the selection's radix histogram
   const int bh = blockIdx.x, tid = threadIdx.x;
   for (int i = tid; i < dm.T; i += 256) E[i] = pp.energy[(size_t)bh * dm.T + i];
   __syncthreads();
-  if (tid < 32) warp_topk(E, dm.T, dm.n_sharp, sharp, bits);
+  if (tid < 32) warp_topk(E, dm.T, dm.n_sharp, sharp, bits, hist);
   __syncthreads();
   for (int i = tid; i < dm.n_sharp; i += 256) pp.sharp[(size_t)bh * dm.n_sharp + i] = sharp[i];
   if (tid < 32) {
@@ -345,6 +347,7 @@ __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
   extern __shared__ float sm[];
   float* qrows = sm;                 // [8][D]
   float* sc = sm + 8 * D;            // [8][T_kv]
+  __shared__ uint32_t hist[8][256];   // each warp's radix histogram
   const int bh = blockIdx.y, f0 = blockIdx.x * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* Qc = pp.Qc + (size_t)bh * dm.T * D;
   const float* Kc = pp.Kc + (size_t)bh * dm.T * D;
@@ -401,7 +404,7 @@ __global__ void __launch_bounds__(256) exact_kernel(Dims dm, PlanPtrs pp) {
   if (f < dm.n_flat) {
     uint32_t* bits = pp.bits + ((size_t)bh * dm.n_flat + f) * dm.words;
     int* ex = pp.exact + ((size_t)bh * dm.n_flat + f) * dm.n_exact;
-    warp_topk(sc + warp * dm.T_kv, dm.T_kv, dm.n_exact, ex, bits);
+    warp_topk(sc + warp * dm.T_kv, dm.T_kv, dm.n_exact, ex, bits, hist[warp]);
   }
 }
 
